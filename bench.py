@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the FlowCache per-step hot path on B200.
+
+One step = the whole hot path over one layer's synthetic inputs, all through
+the libflowcache C-ABI:
+  gate (fused Euler update + per-chunk relative L1 + accumulator) over every
+  chunk, then importance, redundancy, pooled score + top-B, and K/V compaction
+  over every head.
+Default workload: one bf16 layer (H=24, d=128, L_q=4096, L_k=16384, B=8192,
+lambda=0.5, pool 7) with the gate over 4 chunks of 24x45x45x16 fp32 latents
+(T=30, m=5, eps=0.01).
+
+Metric: clean KV tokens scored+selected per second per head (= L_k / step
+time, summed over ranks); the gate's GB/s and each kernel's roofline fraction
+ride along.  Multi-GPU: every rank runs an independent layer (weak scaling,
+no data-path collective); timing is the max over ranks.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "clean KV tokens scored+selected/s per head; L1-gate GB/s; % of roofline"
+UNIT = "tokens/s/head"
+FLUSH_BYTES = 256 << 20  # > 126 MB L2
+# Kernel launches per call, as implemented in cache_gating_kv_b200/csrc.
+LAUNCHES = {"gate": 1, "importance": 2, "redundancy": 3, "score_topb": 2, "compact": 1}
+
+
+def _args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="bf16_layer")
+    ap.add_argument("--cpu-sample-heads", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        p = json.load(open(path))
+        return float(p["hbm_gbs"]), float(p["bf16_tflops"]), float(p["bf16_tflops_sustained"]), \
+            "measured"
+    except Exception:
+        return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = f"/tmp/fc_clocks_{os.getpid()}.csv"
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [s.strip() for s in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        try:
+            os.remove(self.path)
+        except OSError:
+            pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        mhz = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)
+        loaded = [m for m in mhz if mx and m > 0.5 * mx] or mhz
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]})
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# native arm
+# ---------------------------------------------------------------------------
+class Step:
+    """Device buffers of one layer's step and the five C-ABI calls."""
+
+    def __init__(self, kv_cfg, gate_cfg, seed, dev):
+        import cache_gating_kv_b200 as fc
+        from cache_gating_kv_b200 import workloads as W
+
+        self.fc = fc
+        self.kv, self.gc = kv_cfg, gate_cfg
+        q, k, v = W.kv_inputs(kv_cfg, seed=seed)
+        self.host = {"q": q, "k": k, "v": v}
+        x = W.gate_initial(gate_cfg, seed)
+        vel = W.gate_velocity(gate_cfg, seed)
+        gstep = gate_cfg.m + 5 + gate_cfg.stagger * (gate_cfg.n_chunks - 1)
+        st = W.gate_step_counters(gate_cfg, min(gstep, gate_cfg.T - 1))
+        dt = W.gate_dt(gate_cfg, st)
+        self.host.update(x=torch.from_numpy(x), vel=torch.from_numpy(vel),
+                         dt=torch.from_numpy(dt), step=torch.from_numpy(st),
+                         f=torch.zeros(gate_cfg.n_chunks))
+        self.d = {n: t.to(dev) for n, t in self.host.items()}
+        H, Lq, Lk, d, B = kv_cfg.H, kv_cfg.Lq, kv_cfg.Lk, kv_cfg.d, kv_cfg.B
+        code = fc.FC_BF16 if kv_cfg.dtype == "bf16" else fc.FC_F32
+        self.eps = gate_cfg.eps[0]
+        self.lam = kv_cfg.lam[len(kv_cfg.lam) // 2]
+        self.out = {
+            "l1": torch.zeros(gate_cfg.n_chunks, device=dev),
+            "mask": torch.zeros(gate_cfg.n_chunks, dtype=torch.uint8, device=dev),
+            "imp": torch.empty(H, Lk, device=dev), "red": torch.empty(H, Lk, device=dev),
+            "idx": torch.empty(H, B, dtype=torch.int32, device=dev),
+            "ko": torch.empty(H, B, d, dtype=q.dtype, device=dev),
+            "vo": torch.empty(H, B, d, dtype=q.dtype, device=dev),
+        }
+        self.ws = {
+            "gate": fc.workspace(fc.fc_gate_workspace_size(gate_cfg.n_chunks, gate_cfg.N), dev),
+            "imp": fc.workspace(fc.fc_importance_workspace_size(code, H, Lq, Lk, d), dev),
+            "red": fc.workspace(fc.fc_redundancy_workspace_size(code, H, Lk, d), dev),
+            "topb": fc.workspace(fc.fc_score_topb_workspace_size(H, Lk, B), dev),
+        }
+
+    def run(self, stream, ev=None):
+        """Enqueue one step; ``ev`` (6 events) brackets the five calls."""
+        fc, d, o, w = self.fc, self.d, self.out, self.ws
+        if ev:
+            ev[0].record(stream)
+        fc.fc_chunk_l1_gate(d["x"], d["vel"], d["dt"], d["step"], self.gc.m, self.eps, d["f"],
+                            o["l1"], o["mask"], w["gate"], stream=stream)
+        if ev:
+            ev[1].record(stream)
+        fc.fc_kv_importance(d["q"], d["k"], o["imp"], w["imp"], stream=stream)
+        if ev:
+            ev[2].record(stream)
+        fc.fc_kv_redundancy(d["k"], o["red"], w["red"], stream=stream)
+        if ev:
+            ev[3].record(stream)
+        fc.fc_kv_score_topb(o["imp"], o["red"], self.kv.pool, self.lam, self.kv.B, o["idx"],
+                            w["topb"], stream=stream)
+        if ev:
+            ev[4].record(stream)
+        fc.fc_kv_compact(d["k"], d["v"], o["idx"], o["ko"], o["vo"], stream=stream)
+        if ev:
+            ev[5].record(stream)
+
+    def reset_gate(self):
+        self.d["x"].copy_(self.host["x"])
+        self.d["f"].zero_()
+
+
+def _bytes_gate(gc):
+    return 12 * gc.n_chunks * gc.N
+
+
+def native(a, rank, world, local_rank):
+    from cache_gating_kv_b200 import workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    kv_cfg, gate_cfg = W.KV_CONFIGS[a.workload], W.GATE_CONFIGS[a.workload]
+    step = Step(kv_cfg, gate_cfg, seed=rank, dev=dev)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    names = ["gate", "importance", "redundancy", "score_topb", "compact"]
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    with torch.cuda.stream(stream):
+        for _ in range(a.warmup):
+            flush.zero_()
+            step.run(stream)
+        stream.synchronize()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(a.steps)]
+        clocks = Clocks(local_rank)
+        barrier()
+        torch.cuda.synchronize()
+        clocks.start()
+        for i in range(a.steps):
+            flush.zero_()  # L2 flush between steps, outside the timed events
+            step.run(stream, evs[i])
+        stream.synchronize()
+        torch.cuda.synchronize()
+        barrier()
+        ck = clocks.stop()
+    per = {n: [] for n in names}
+    tot = []
+    for e in evs:
+        for j, n in enumerate(names):
+            per[n].append(e[j].elapsed_time(e[j + 1]))
+        tot.append(e[0].elapsed_time(e[5]))
+    ms_step = sum(tot) / len(tot)
+    ms_call = {n: sum(v) / len(v) for n, v in per.items()}
+
+    # end to end through the public API with host buffers (pinned), every step
+    e2e = None
+    if not a.no_e2e:
+        e2e = _e2e(step, stream, flush, a, dev)
+
+    t_max = ms_step
+    if world > 1:
+        t = torch.tensor([ms_step] + ([e2e["ms"]] if e2e else []), device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_max = float(t[0])
+        if e2e:
+            e2e["ms"] = float(t[1])
+    H, Lq, Lk, d = kv_cfg.H, kv_cfg.Lq, kv_cfg.Lk, kv_cfg.d
+    value = world * Lk / (t_max * 1e-3)  # tokens/s per head over all ranks
+    hbm, tf_burst, tf_sus, src = _peaks()
+    exec_flops = 4.0 * H * Lq * Lk * d  # two passes of Q K^T
+    imp_tf = exec_flops / (ms_call["importance"] * 1e-3) / 1e12
+    gate_gbs = _bytes_gate(gate_cfg) / (ms_call["gate"] * 1e-3) / 1e9
+    elem = 2 if kv_cfg.dtype == "bf16" else 4
+    red_gbs = H * Lk * d * elem / (ms_call["redundancy"] * 1e-3) / 1e9
+    comp_gbs = 2 * 2 * H * kv_cfg.B * d * elem / (ms_call["compact"] * 1e-3) / 1e9
+    topb_gbs = H * Lk * 12 / (ms_call["score_topb"] * 1e-3) / 1e9
+    launches = sum(LAUNCHES.values()) * a.steps
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": t_max, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": kv_cfg.dtype if kv_cfg.dtype == "bf16" else "f32",
+        "data": "synthetic (seeded AR(1) keys, N(0,1) queries/values, flow-matching toy latents)",
+        "config": {"workload": f"{a.workload}: H={H} d={d} L_q={Lq} L_k={Lk} B={kv_cfg.B} "
+                               f"lambda={step.lam} pool={kv_cfg.pool}; gate {gate_cfg.n_chunks}x"
+                               f"{gate_cfg.N} fp32 m={gate_cfg.m} eps={step.eps}",
+                   "per_rank": "one independent layer per GPU",
+                   "l2": "flushed between steps (256 MiB write, outside the timed events)"},
+        "roofline": {"bound": "tensor", "kernel": "fc_kv_importance (2 passes)",
+                     "achieved": imp_tf, "peak": tf_burst, "unit": "TFLOP/s",
+                     "frac": imp_tf / tf_burst, "peak_source": f"{src} bf16 burst",
+                     "flops_per_launch": exec_flops, "traffic": None},
+        "kernels_ms": ms_call,
+        "gate": {"GB/s": gate_gbs, "frac_hbm": gate_gbs / hbm},
+        "redundancy": {"GB/s": red_gbs, "frac_hbm": red_gbs / hbm},
+        "score_topb": {"GB/s": topb_gbs},
+        "compact": {"GB/s": comp_gbs, "frac_hbm": comp_gbs / hbm},
+        "gpu_launches": launches,
+        "clocks": ck,
+    }
+    if e2e:
+        out["e2e"] = {"value": world * Lk / (e2e["ms"] * 1e-3), "unit": UNIT,
+                      "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
+    return out
+
+
+def _e2e(step, stream, flush, a, dev):
+    """Same step with pinned host inputs copied in and the results read back,
+    inside the timed region, every step."""
+    host_in = {n: t.pin_memory() for n, t in step.host.items()}
+    res = ["l1", "mask", "idx"]
+    host_out = {n: torch.empty_like(step.out[n], device="cpu").pin_memory() for n in res}
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values()) + \
+        step.d["f"].numel() * 4
+    host_f = torch.empty_like(step.host["f"]).pin_memory()
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(a.warmup + a.steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for n, t in host_in.items():
+                step.d[n].copy_(t, non_blocking=True)
+            step.run(stream)
+            for n in res:
+                host_out[n].copy_(step.out[n], non_blocking=True)
+            host_f.copy_(step.d["f"], non_blocking=True)
+            e1.record(stream)
+            e1.synchronize()
+            if i >= a.warmup:
+                times.append(e0.elapsed_time(e1))
+    return {"ms": sum(times) / len(times), "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle legs
+# ---------------------------------------------------------------------------
+def _oracle_step_seconds(kv_cfg, gate_cfg, heads, seed=0):
+    """Oracle time for the compression of ``heads`` heads plus one full gate step."""
+    from cache_gating_kv_b200 import workloads as W
+    from oracle import flowcache_oracle as O
+
+    q, k, v = W.kv_inputs(kv_cfg, seed=seed, heads=list(range(heads)))
+    q64 = q.float().numpy().astype(np.float64)
+    k64 = k.float().numpy().astype(np.float64)
+    kf, vf = k.float().numpy(), v.float().numpy()
+    x = W.gate_initial(gate_cfg, seed)
+    vel = W.gate_velocity(gate_cfg, seed)
+    st = W.gate_step_counters(gate_cfg, gate_cfg.m + 5)
+    dt = W.gate_dt(gate_cfg, st)
+    lam = kv_cfg.lam[len(kv_cfg.lam) // 2]
+    t0 = time.perf_counter()
+    O.gate_step(x, vel, dt, st, gate_cfg.m, gate_cfg.eps[0], np.zeros(gate_cfg.n_chunks, np.float32))
+    t1 = time.perf_counter()
+    imp = O.importance(q64, k64)
+    red = O.redundancy(k64)
+    _, idx = O.score_topb(imp, red, lam, kv_cfg.pool, kv_cfg.B)
+    O.compact(kf, vf, idx)
+    t2 = time.perf_counter()
+    return t1 - t0, (t2 - t1) / heads
+
+
+def _cores():
+    try:
+        from threadpoolctl import threadpool_info
+        return max(int(i.get("num_threads", 1)) for i in threadpool_info()) or os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(a):
+    from cache_gating_kv_b200 import workloads as W
+
+    kv_cfg, gate_cfg = W.KV_CONFIGS[a.workload], W.GATE_CONFIGS[a.workload]
+    heads = max(1, min(a.cpu_sample_heads, kv_cfg.H))
+    t_gate, t_head = _oracle_step_seconds(kv_cfg, gate_cfg, heads)
+    t_step = t_gate + kv_cfg.H * t_head
+    return {"value": kv_cfg.Lk / t_step, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+            "sample": f"{heads} of {kv_cfg.H} heads of the compression (importance, redundancy, "
+                      f"score/top-B, compaction) plus one full gate step; step time = gate + "
+                      f"H x per-head time"}
+
+
+def reference(a, rank):
+    if rank != 0:
+        return None
+    from cache_gating_kv_b200 import workloads as W
+
+    kv_cfg, gate_cfg = W.KV_CONFIGS[a.workload], W.GATE_CONFIGS[a.workload]
+    times = []
+    for i in range(a.warmup + a.steps):
+        t_gate, t_head = _oracle_step_seconds(kv_cfg, gate_cfg, 1, seed=i)
+        if i >= a.warmup:
+            times.append(t_gate + kv_cfg.H * t_head)
+    t = sum(times) / len(times)
+    value = kv_cfg.Lk / t
+    sample = ("each step: 1 of the layer's heads through the oracle's compression plus one "
+              "full gate step; step time = gate + H x per-head time")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": t * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic",
+            "config": {"workload": a.workload},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    a = _args()
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if a.impl == "reference":
+        out = reference(a, rank)
+        if out is not None:
+            print(json.dumps(out))
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        out = native(a, rank, world, local_rank)
+        if rank == 0:
+            if not a.no_cpu_baseline:
+                out["cpu_baseline"] = cpu_baseline(a)
+            print(json.dumps(out))
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

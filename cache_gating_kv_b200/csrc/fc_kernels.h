@@ -1,0 +1,43 @@
+// Internal launchers of libflowcache.  Each returns the CUDA error of its
+// launches (cudaSuccess when everything was enqueued).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace fc {
+
+// ---- chunkwise gate --------------------------------------------------------
+size_t gate_ws_bytes(int n_chunks);
+cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
+                        const float* dt, const int32_t* step, int m, float eps, float* f,
+                        float* l1, uint8_t* mask, void* ws, cudaStream_t s);
+
+// ---- importance --------------------------------------------------------------
+size_t importance_ws_bytes(int H, int Lq);
+// bf16 tensor-core path (tcgen05 + TMEM + TMA)
+cudaError_t launch_importance_tc(const void* q, const void* k, int H, int Lq, int Lk, int d,
+                                 float scale, float* imp, void* ws, cudaStream_t s);
+bool importance_tc_supported(int d);
+// CUDA-core path (float32 or bf16 inputs)
+cudaError_t launch_importance_simt(const void* q, const void* k, bool bf16, int H, int Lq,
+                                   int Lk, int d, float scale, float* imp, void* ws,
+                                   cudaStream_t s);
+
+// ---- redundancy ----------------------------------------------------------------
+size_t redundancy_ws_bytes(int H, int d);
+cudaError_t launch_redundancy(const void* k, bool bf16, int H, int Lk, int d, float* red,
+                              void* ws, cudaStream_t s);
+
+// ---- score + top-B ---------------------------------------------------------------
+size_t score_topb_ws_bytes(int H, int Lk);
+cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk, int pool,
+                              float lambda, int B, float* score, int32_t* idx, void* ws,
+                              cudaStream_t s);
+
+// ---- compaction ------------------------------------------------------------------
+cudaError_t launch_compact(const void* k, const void* v, int elem_bytes, int H, int Lk, int d,
+                           const int32_t* idx, int B, void* k_out, void* v_out, cudaStream_t s);
+
+}  // namespace fc

@@ -1,0 +1,221 @@
+// C-ABI of libflowcache: argument validation on the host, then launches.
+// The declarations and their contracts are in include/flowcache.h.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "../../include/flowcache.h"
+#include "fc_common.cuh"
+#include "fc_kernels.h"
+
+namespace fc {
+
+int sm_count() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace fc
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+fc_status fail(fc_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+fc_status ok() {
+  g_err[0] = '\0';
+  return FC_OK;
+}
+
+// Null, misalignment and host-memory checks for one tensor argument.
+fc_status check_ptr(const void* p, const char* name) {
+  if (p == nullptr) return fail(FC_ERR_INVALID_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(p) % 16 != 0)
+    return fail(FC_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  cudaPointerAttributes a;
+  const cudaError_t e = cudaPointerGetAttributes(&a, p);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(FC_ERR_CUDA, "cudaPointerGetAttributes(%s): %s", name, cudaGetErrorString(e));
+  }
+  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged)
+    return fail(FC_ERR_INVALID_ARG, "%s is not device memory", name);
+  return FC_OK;
+}
+
+#define FC_CHECK_PTR(p)                        \
+  do {                                         \
+    fc_status _st = check_ptr((p), #p);        \
+    if (_st != FC_OK) return _st;              \
+  } while (0)
+
+fc_status launched(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(FC_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+  return ok();
+}
+
+size_t elem_bytes(fc_dtype t) { return t == FC_BF16 ? 2 : 4; }
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+  const char* pa = static_cast<const char*>(a);
+  const char* pb = static_cast<const char*>(b);
+  return pa < pb + nb && pb < pa + na;
+}
+
+fc_status check_kv_shape(fc_dtype dtype, int H, int L1, int L2, int d) {
+  if (dtype != FC_F32 && dtype != FC_BF16) return fail(FC_ERR_INVALID_ARG, "unknown dtype %d", (int)dtype);
+  if (H < 1 || L1 < 1 || L2 < 1) return fail(FC_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (H > 65535) return fail(FC_ERR_INVALID_ARG, "H must be <= 65535");
+  if (d != 64 && d != 128) return fail(FC_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+  return FC_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fc_last_error(void) { return g_err; }
+
+int fc_version(void) { return 100; }
+
+size_t fc_gate_workspace_size(int n_chunks, int64_t n_per_chunk) {
+  (void)n_per_chunk;
+  return n_chunks < 1 ? 0 : fc::gate_ws_bytes(n_chunks);
+}
+
+fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
+                           const float* dt, const int32_t* step, int32_t m, float eps, float* f,
+                           float* l1_rel, uint8_t* recompute, void* ws, size_t ws_bytes,
+                           void* stream) {
+  if (n_chunks < 1 || n_chunks > 65535)
+    return fail(FC_ERR_INVALID_ARG, "n_chunks must be in [1, 65535] (got %d)", n_chunks);
+  if (n_per_chunk < 0) return fail(FC_ERR_INVALID_ARG, "n_per_chunk must be >= 0");
+  if (m < 0) return fail(FC_ERR_INVALID_ARG, "m must be >= 0");
+  if (ws == nullptr || ws_bytes < fc::gate_ws_bytes(n_chunks))
+    return fail(FC_ERR_WORKSPACE, "gate workspace needs %zu bytes", fc::gate_ws_bytes(n_chunks));
+  FC_CHECK_PTR(x);
+  FC_CHECK_PTR(v);
+  FC_CHECK_PTR(dt);
+  FC_CHECK_PTR(step);
+  FC_CHECK_PTR(f);
+  FC_CHECK_PTR(l1_rel);
+  FC_CHECK_PTR(recompute);
+  FC_CHECK_PTR(ws);
+  return launched(fc::launch_gate(x, v, n_chunks, n_per_chunk, dt, step, m, eps, f, l1_rel,
+                                  recompute, ws, static_cast<cudaStream_t>(stream)),
+                  "fc_chunk_l1_gate");
+}
+
+size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d) {
+  (void)dtype;
+  (void)Lk;
+  (void)d;
+  return (H < 1 || Lq < 1) ? 0 : fc::importance_ws_bytes(H, Lq);
+}
+
+fc_status fc_kv_importance(const void* q, const void* k, fc_dtype dtype, int H, int Lq, int Lk,
+                           int d, float scale, float* imp, void* ws, size_t ws_bytes,
+                           void* stream) {
+  fc_status st = check_kv_shape(dtype, H, Lq, Lk, d);
+  if (st != FC_OK) return st;
+  if (ws == nullptr || ws_bytes < fc::importance_ws_bytes(H, Lq))
+    return fail(FC_ERR_WORKSPACE, "importance workspace needs %zu bytes",
+                fc::importance_ws_bytes(H, Lq));
+  FC_CHECK_PTR(q);
+  FC_CHECK_PTR(k);
+  FC_CHECK_PTR(imp);
+  FC_CHECK_PTR(ws);
+  if (!(scale > 0.0f)) scale = 1.0f / sqrtf((float)d);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (dtype == FC_BF16 && fc::importance_tc_supported(d))
+    return launched(fc::launch_importance_tc(q, k, H, Lq, Lk, d, scale, imp, ws, s),
+                    "fc_kv_importance");
+  return launched(fc::launch_importance_simt(q, k, dtype == FC_BF16, H, Lq, Lk, d, scale, imp,
+                                             ws, s),
+                  "fc_kv_importance");
+}
+
+size_t fc_redundancy_workspace_size(fc_dtype dtype, int H, int Lk, int d) {
+  (void)dtype;
+  (void)Lk;
+  return (H < 1 || (d != 64 && d != 128)) ? 0 : fc::redundancy_ws_bytes(H, d);
+}
+
+fc_status fc_kv_redundancy(const void* k, fc_dtype dtype, int H, int Lk, int d, float* red,
+                           void* ws, size_t ws_bytes, void* stream) {
+  fc_status st = check_kv_shape(dtype, H, Lk, Lk, d);
+  if (st != FC_OK) return st;
+  if (ws == nullptr || ws_bytes < fc::redundancy_ws_bytes(H, d))
+    return fail(FC_ERR_WORKSPACE, "redundancy workspace needs %zu bytes",
+                fc::redundancy_ws_bytes(H, d));
+  FC_CHECK_PTR(k);
+  FC_CHECK_PTR(red);
+  FC_CHECK_PTR(ws);
+  return launched(fc::launch_redundancy(k, dtype == FC_BF16, H, Lk, d, red, ws,
+                                        static_cast<cudaStream_t>(stream)),
+                  "fc_kv_redundancy");
+}
+
+size_t fc_score_topb_workspace_size(int H, int Lk, int B) {
+  (void)B;
+  return (H < 1 || Lk < 1) ? 0 : fc::score_topb_ws_bytes(H, Lk);
+}
+
+fc_status fc_kv_score_topb(const float* imp, const float* red, int H, int Lk, int pool_window,
+                           float lambda, int B, float* score, int32_t* idx, void* ws,
+                           size_t ws_bytes, void* stream) {
+  if (H < 1 || H > 65535 || Lk < 1) return fail(FC_ERR_INVALID_ARG, "H and Lk must be >= 1");
+  if (B < 1) return fail(FC_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
+  if (pool_window < 1 || pool_window % 2 == 0 || pool_window > 511)
+    return fail(FC_ERR_INVALID_ARG, "pool_window must be odd and in [1, 511] (got %d)",
+                pool_window);
+  if (ws == nullptr || ws_bytes < fc::score_topb_ws_bytes(H, Lk))
+    return fail(FC_ERR_WORKSPACE, "score/top-B workspace needs %zu bytes",
+                fc::score_topb_ws_bytes(H, Lk));
+  FC_CHECK_PTR(imp);
+  FC_CHECK_PTR(red);
+  FC_CHECK_PTR(idx);
+  FC_CHECK_PTR(ws);
+  if (score != nullptr) FC_CHECK_PTR(score);
+  return launched(fc::launch_score_topb(imp, red, H, Lk, pool_window, lambda, B, score, idx, ws,
+                                        static_cast<cudaStream_t>(stream)),
+                  "fc_kv_score_topb");
+}
+
+fc_status fc_kv_compact(const void* k, const void* v, fc_dtype dtype, int H, int Lk, int d,
+                        const int32_t* idx, int B, void* k_out, void* v_out, void* stream) {
+  fc_status st = check_kv_shape(dtype, H, Lk, Lk, d);
+  if (st != FC_OK) return st;
+  if (B < 1) return fail(FC_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
+  FC_CHECK_PTR(k);
+  FC_CHECK_PTR(v);
+  FC_CHECK_PTR(idx);
+  FC_CHECK_PTR(k_out);
+  FC_CHECK_PTR(v_out);
+  const size_t in_bytes = (size_t)H * Lk * d * elem_bytes(dtype);
+  const size_t out_bytes = (size_t)H * B * d * elem_bytes(dtype);
+  if (ranges_overlap(k_out, out_bytes, k, in_bytes) || ranges_overlap(k_out, out_bytes, v, in_bytes) ||
+      ranges_overlap(v_out, out_bytes, k, in_bytes) || ranges_overlap(v_out, out_bytes, v, in_bytes) ||
+      ranges_overlap(k_out, out_bytes, v_out, out_bytes))
+    return fail(FC_ERR_INVALID_ARG, "k_out / v_out overlap an input or each other");
+  return launched(fc::launch_compact(k, v, (int)elem_bytes(dtype), H, Lk, d, idx, B, k_out, v_out,
+                                     static_cast<cudaStream_t>(stream)),
+                  "fc_kv_compact");
+}
+
+}  // extern "C"

@@ -1,0 +1,199 @@
+// Chunkwise cache gate: fused Euler update, per-chunk relative-L1 reduction
+// and the accumulator recurrence, in one memory-bound pass.
+//
+// Method: "Flow Caching for Autoregressive Video Generation" (papernotes.org),
+// 方法详解 / 关键设计 1 (L1_rel = ||v*dt||_1 / ||X_t||_1, the update form of the
+// relative L1 distance between X_{t-1} and X_t) and 关键设计 2 (per-chunk
+// accumulator f: forced recompute for the first m steps, recompute and reset
+// when f + L1_rel > eps, otherwise accumulate and reuse).
+//
+// Design (B200): the pass moves 12 bytes per element (read X, read v, write
+// X), so it is bound by HBM.  The grid is n_chunks x blocks_per_chunk with the
+// total sized to fill all SMs; every thread streams 16-byte vectors with
+// read-once cache hints, unrolled so that each thread keeps eight loads in
+// flight.  Partial sums are float64 (exact enough that the float32 L1_rel is
+// practically the correctly rounded quotient).  Each block stores its partial
+// pair; the last block of a chunk to finish (an integer completion counter,
+// no spinning, no float atomics) sums the partials in a fixed order and runs
+// the recurrence, so the result is deterministic and one launch does it all.
+#include "fc_common.cuh"
+#include "fc_kernels.h"
+
+namespace fc {
+
+namespace {
+constexpr int kGateThreads = 256;
+constexpr int kGateUnroll = 4;
+constexpr int kGateMaxBlocksPerChunk = 1024;
+
+__device__ __forceinline__ void gate_finalize(int c, int st, int m, float eps, double num,
+                                              double den, float* f, float* l1, uint8_t* mask) {
+  float r;
+  if (den > 0.0)
+    r = (float)(num / den);
+  else
+    r = (num > 0.0) ? __int_as_float(0x7f800000) : 0.0f;
+  l1[c] = r;
+  if (st < m) {  // forced recompute during the first m steps of the chunk
+    mask[c] = 1;
+    f[c] = 0.0f;
+  } else {
+    const float acc = __fadd_rn(f[c], r);
+    if (acc > eps) {  // recompute and reset
+      mask[c] = 1;
+      f[c] = 0.0f;
+    } else {  // reuse, accumulate
+      mask[c] = 0;
+      f[c] = acc;
+    }
+  }
+}
+
+__device__ __forceinline__ void gate_elem(float& x, float vv, float h, double& num, double& den) {
+  const float p = __fmul_rn(vv, h);  // v*dt, rounded once
+  num += (double)fabsf(p);
+  den += (double)fabsf(x);
+  x = __fadd_rn(x, p);  // X_{t-1} = X_t + v*dt, rounded once
+}
+
+__global__ void __launch_bounds__(kGateThreads)
+    gate_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t N,
+                const float* __restrict__ dt, const int32_t* __restrict__ step, int m, float eps,
+                float* __restrict__ f, float* __restrict__ l1, uint8_t* __restrict__ mask,
+                unsigned* __restrict__ counters, double2* __restrict__ partials, int bpc) {
+  const int c = blockIdx.y;
+  const int b = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int st = step[c];
+  if (st < 0) {  // inactive chunk: nothing touched
+    if (b == 0 && tid == 0) {
+      l1[c] = 0.0f;
+      mask[c] = 0;
+    }
+    return;
+  }
+  const float h = dt[c];
+  const int64_t off = (int64_t)c * N;
+  float* xc = x + off;
+  const float* vc = v + off;
+
+  // x and v are 16-byte aligned, so the chunk's misalignment is off mod 4.
+  const int64_t mis = off & 3;
+  int64_t head = mis ? 4 - mis : 0;
+  if (head > N) head = N;
+  const int64_t nvec = (N - head) >> 2;
+  const int64_t tail0 = head + (nvec << 2);
+
+  const int64_t per = ceil_div(nvec, bpc);
+  const int64_t lo = min(nvec, per * b);
+  const int64_t hi = min(nvec, lo + per);
+  float4* x4 = reinterpret_cast<float4*>(xc + head);
+  const float4* v4 = reinterpret_cast<const float4*>(vc + head);
+
+  double num = 0.0, den = 0.0;
+  for (int64_t base = lo + tid; base < hi; base += (int64_t)kGateThreads * kGateUnroll) {
+    float4 xa[kGateUnroll], va[kGateUnroll];
+#pragma unroll
+    for (int u = 0; u < kGateUnroll; ++u) {
+      const int64_t i = base + (int64_t)u * kGateThreads;
+      if (i < hi) {
+        xa[u] = __ldcs(x4 + i);
+        va[u] = __ldcs(v4 + i);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kGateUnroll; ++u) {
+      const int64_t i = base + (int64_t)u * kGateThreads;
+      if (i < hi) {
+        gate_elem(xa[u].x, va[u].x, h, num, den);
+        gate_elem(xa[u].y, va[u].y, h, num, den);
+        gate_elem(xa[u].z, va[u].z, h, num, den);
+        gate_elem(xa[u].w, va[u].w, h, num, den);
+        __stcs(x4 + i, xa[u]);
+      }
+    }
+  }
+  // Unaligned head (< 4 elements) and tail (< 4 elements): block 0.
+  if (b == 0) {
+    int64_t e = -1;
+    if (tid < head)
+      e = tid;
+    else if (tid >= 4 && tid - 4 < N - tail0)
+      e = tail0 + (tid - 4);
+    if (e >= 0) {
+      float xv = xc[e];
+      gate_elem(xv, vc[e], h, num, den);
+      xc[e] = xv;
+    }
+  }
+
+  // Block reduction in a fixed order.
+  __shared__ double s_num[kGateThreads / 32], s_den[kGateThreads / 32];
+  __shared__ int s_last;
+  num = warp_sum(num);
+  den = warp_sum(den);
+  const int warp = tid >> 5, lane = tid & 31;
+  if (lane == 0) {
+    s_num[warp] = num;
+    s_den[warp] = den;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    double a = 0.0, d = 0.0;
+#pragma unroll
+    for (int w = 0; w < kGateThreads / 32; ++w) {
+      a += s_num[w];
+      d += s_den[w];
+    }
+    partials[(size_t)c * kGateMaxBlocksPerChunk + b] = make_double2(a, d);
+    __threadfence();  // publish the partial before counting this block done
+    const unsigned prev = atomicAdd(&counters[c], 1u);
+    s_last = (prev == (unsigned)(bpc - 1));
+  }
+  __syncthreads();
+  if (!s_last) return;
+
+  // Last block of chunk c: fixed-order sum of every block's partial.
+  __threadfence();
+  if (warp == 0) {
+    double a = 0.0, d = 0.0;
+    for (int i = lane; i < bpc; i += 32) {
+      const double2 p = __ldcg(&partials[(size_t)c * kGateMaxBlocksPerChunk + i]);
+      a += p.x;
+      d += p.y;
+    }
+    a = warp_sum(a);
+    d = warp_sum(d);
+    if (lane == 0) {
+      gate_finalize(c, st, m, eps, a, d, f, l1, mask);
+      counters[c] = 0u;  // ready for the next call
+    }
+  }
+}
+}  // namespace
+
+size_t gate_ws_bytes(int n_chunks) {
+  return align_up((size_t)n_chunks * sizeof(unsigned), 256) +
+         (size_t)n_chunks * kGateMaxBlocksPerChunk * sizeof(double2);
+}
+
+cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t N, const float* dt,
+                        const int32_t* step, int m, float eps, float* f, float* l1,
+                        uint8_t* mask, void* ws, cudaStream_t s) {
+  unsigned* counters = static_cast<unsigned*>(ws);
+  double2* partials = reinterpret_cast<double2*>(static_cast<char*>(ws) +
+                                                 align_up((size_t)n_chunks * 4, 256));
+  // Four resident 256-thread blocks per SM over the whole grid.
+  const int64_t target = (int64_t)sm_count() * 4;
+  int64_t bpc = ceil_div(target, n_chunks);
+  const int64_t useful = ceil_div(N / 4 + 1, kGateThreads);  // >= one vector per thread
+  if (bpc > useful) bpc = useful;
+  if (bpc < 1) bpc = 1;
+  if (bpc > kGateMaxBlocksPerChunk) bpc = kGateMaxBlocksPerChunk;
+  dim3 grid((unsigned)bpc, (unsigned)n_chunks);
+  gate_kernel<<<grid, kGateThreads, 0, s>>>(x, v, N, dt, step, m, eps, f, l1, mask, counters,
+                                            partials, (int)bpc);
+  return cudaGetLastError();
+}
+
+}  // namespace fc

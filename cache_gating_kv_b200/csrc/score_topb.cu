@@ -1,0 +1,233 @@
+// Joint score and per-head top-B selection.
+//
+// Method: "Flow Caching for Autoregressive Video Generation" (papernotes.org),
+// 方法详解 / 关键设计 3: Imp~ is the 1D max-pooled importance;
+// Score_j = lambda*Imp~_j - (1-lambda)*Red_j; each head keeps its top-B tokens.
+//
+//   score kernel   grid (L_k/1024, H): pooled importance from a shared-memory
+//                  tile with halo, the float32 score, and an order-preserving
+//                  uint32 key (larger score -> larger key; -0 folded into +0)
+//   select kernel  one 1024-thread block per head: a 4-pass MSB radix select
+//                  (8-bit digits, per-warp histograms with match_any
+//                  aggregation) finds the B-th largest key T and how many
+//                  copies of T to keep; then one ordered compaction pass writes
+//                  every kept index, ascending, using warp ballots for the
+//                  in-warp ranks and a block scan over warps.  Ties at T keep
+//                  the lowest indices.
+// Keys are staged in shared memory when a head's keys fit, otherwise they are
+// re-read from global memory (L2-resident) on every pass.
+#include "fc_common.cuh"
+#include "fc_kernels.h"
+
+namespace fc {
+
+namespace {
+constexpr int kScoreTile = 1024;
+constexpr int kScoreThreads = 256;
+constexpr int kSelThreads = 1024;
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kMaxPool = 255;
+constexpr int kHistBytes = kSelWarps * 256 * 4;
+constexpr int kSelSmemLimit = 220 * 1024;
+
+__device__ __forceinline__ uint32_t order_key(float s) {
+  uint32_t u = __float_as_uint(s);
+  if (u == 0x80000000u) u = 0u;  // -0 ties with +0
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__global__ void __launch_bounds__(kScoreThreads)
+    score_kernel(const float* __restrict__ imp, const float* __restrict__ red, int Lk, int r,
+                 float lam, float one_minus_lam, float* __restrict__ score,
+                 uint32_t* __restrict__ keys) {
+  __shared__ float tile[kScoreTile + 2 * kMaxPool];
+  const int h = blockIdx.y;
+  const int j0 = blockIdx.x * kScoreTile;
+  const float* ih = imp + (size_t)h * Lk;
+  const int n = kScoreTile + 2 * r;
+  for (int t = threadIdx.x; t < n; t += kScoreThreads) {
+    const int j = j0 - r + t;
+    tile[t] = (j >= 0 && j < Lk) ? ih[j] : -INFINITY;  // out-of-range taps ignored
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < kScoreTile; t += kScoreThreads) {
+    const int j = j0 + t;
+    if (j >= Lk) break;
+    float p = tile[t];
+    for (int o = 1; o <= 2 * r; ++o) p = fmaxf(p, tile[t + o]);
+    const float a = __fmul_rn(lam, p);
+    const float b = __fmul_rn(one_minus_lam, red[(size_t)h * Lk + j]);
+    const float sc = __fsub_rn(a, b);
+    if (score) score[(size_t)h * Lk + j] = sc;
+    keys[(size_t)h * Lk + j] = order_key(sc);
+  }
+}
+
+template <bool kStaged>
+__global__ void __launch_bounds__(kSelThreads)
+    select_kernel(const uint32_t* __restrict__ keys, int Lk, int B, int32_t* __restrict__ idx) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  unsigned* hist = reinterpret_cast<unsigned*>(smem);  // [kSelWarps][256]
+  uint32_t* skeys = reinterpret_cast<uint32_t*>(smem + kHistBytes);
+  __shared__ unsigned s_total[256];
+  __shared__ uint32_t s_prefix, s_pmask;
+  __shared__ int s_remaining;
+  __shared__ int s_gt[kSelWarps], s_tie[kSelWarps];
+
+  const int h = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t* kh = keys + (size_t)h * Lk;
+  if (kStaged) {
+    for (int j = tid; j < Lk; j += kSelThreads) skeys[j] = kh[j];
+  }
+  auto key_at = [&](int j) -> uint32_t { return kStaged ? skeys[j] : __ldcg(kh + j); };
+  if (tid == 0) {
+    s_prefix = 0u;
+    s_pmask = 0u;
+    s_remaining = B;
+  }
+
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int i = tid; i < kSelWarps * 256; i += kSelThreads) hist[i] = 0u;
+    __syncthreads();
+    const uint32_t prefix = s_prefix, pmask = s_pmask;
+    unsigned* wh = hist + warp * 256;
+    for (int j0 = warp * 32; j0 < Lk; j0 += kSelThreads) {
+      const int j = j0 + lane;
+      uint32_t key = 0u;
+      bool in = false;
+      if (j < Lk) {
+        key = key_at(j);
+        in = (key & pmask) == prefix;
+      }
+      const unsigned vm = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const unsigned digit = (key >> shift) & 0xffu;
+        const unsigned peers = __match_any_sync(vm, digit);
+        if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&wh[digit], __popc(peers));
+      }
+    }
+    __syncthreads();
+    if (tid < 256) {
+      unsigned t = 0u;
+#pragma unroll 8
+      for (int w = 0; w < kSelWarps; ++w) t += hist[w * 256 + tid];
+      s_total[tid] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // Lane l owns bins 255-8l .. 248-8l (lane 0 the largest digits).
+      const int top = 255 - 8 * lane;
+      unsigned mine = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mine += s_total[top - i];
+      unsigned cum = mine;  // inclusive scan from lane 0
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, cum, o);
+        if (lane >= o) cum += y;
+      }
+      const unsigned need = (unsigned)s_remaining;
+      const unsigned hit = __ballot_sync(0xffffffffu, cum >= need);
+      const int L = __ffs(hit) - 1;  // exists: the prefix holds >= need keys
+      if (lane == L) {
+        unsigned before = cum - mine;
+        int digit = top;
+        for (int i = 0; i < 8; ++i) {
+          const unsigned c = s_total[top - i];
+          if (before + c >= need) {
+            digit = top - i;
+            break;
+          }
+          before += c;
+        }
+        s_remaining = (int)(need - before);
+        s_prefix = s_prefix | ((uint32_t)digit << shift);
+        s_pmask = s_pmask | (0xffu << shift);
+      }
+    }
+    __syncthreads();
+  }
+
+  // T = the B-th largest key; keep every key > T and the first `need` keys == T.
+  const uint32_t T = s_prefix;
+  const int need = s_remaining;
+  const int seg = (int)ceil_div(ceil_div(Lk, kSelWarps), 32) * 32;
+  const int w_lo = min(Lk, warp * seg), w_hi = min(Lk, w_lo + seg);
+  int gt = 0, tie = 0;
+  for (int j0 = w_lo; j0 < w_hi; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < w_hi ? key_at(j) : 0u;
+    gt += __popc(__ballot_sync(0xffffffffu, j < w_hi && key > T));
+    tie += __popc(__ballot_sync(0xffffffffu, j < w_hi && key == T));
+  }
+  if (lane == 0) {
+    s_gt[warp] = gt;
+    s_tie[warp] = tie;
+  }
+  __syncthreads();
+  int gt_base = 0, tie_base = 0;
+  for (int w = 0; w < warp; ++w) {
+    gt_base += s_gt[w];
+    tie_base += s_tie[w];
+  }
+  int out = gt_base + min(need, tie_base);  // kept indices before this warp
+  int tie_run = tie_base;
+  const unsigned lt = (1u << lane) - 1u;
+  int32_t* oh = idx + (size_t)h * B;
+  for (int j0 = w_lo; j0 < w_hi; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < w_hi ? key_at(j) : 0u;
+    const bool is_gt = j < w_hi && key > T;
+    const bool is_tie = j < w_hi && key == T;
+    const unsigned tb = __ballot_sync(0xffffffffu, is_tie);
+    const bool sel = is_gt || (is_tie && tie_run + __popc(tb & lt) < need);
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    const int pos = out + __popc(sb & lt);
+    if (sel && pos < B) oh[pos] = j;  // pos < B always holds; the check keeps writes in bounds
+    out += __popc(sb);
+    tie_run += __popc(tb);
+  }
+}
+
+__global__ void fill_all_kernel(int32_t* idx, int Lk, int B, int H) {
+  const int64_t n = (int64_t)H * B;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int r = (int)(i % B);
+    idx[i] = r < Lk ? r : -1;
+  }
+}
+}  // namespace
+
+size_t score_topb_ws_bytes(int H, int Lk) { return align_up((size_t)H * Lk * 4, 256); }
+
+cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk, int pool,
+                              float lambda, int B, float* score, int32_t* idx, void* ws,
+                              cudaStream_t s) {
+  uint32_t* keys = static_cast<uint32_t*>(ws);
+  const float one_minus = 1.0f - lambda;  // float32, as the score's definition
+  dim3 g1((unsigned)ceil_div(Lk, kScoreTile), H);
+  score_kernel<<<g1, kScoreThreads, 0, s>>>(imp, red, Lk, pool / 2, lambda, one_minus, score,
+                                            keys);
+  if (B >= Lk) {
+    const int64_t nfb = ceil_div((int64_t)H * B, 256);
+    fill_all_kernel<<<(unsigned)(nfb < 1024 ? nfb : 1024), 256, 0, s>>>(
+        idx, Lk, B, H);
+    return cudaGetLastError();
+  }
+  const size_t staged = (size_t)kHistBytes + (size_t)Lk * 4;
+  if (staged <= (size_t)kSelSmemLimit) {
+    cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)staged);
+    select_kernel<true><<<H, kSelThreads, staged, s>>>(keys, Lk, B, idx);
+  } else {
+    cudaFuncSetAttribute(select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         kHistBytes);
+    select_kernel<false><<<H, kSelThreads, kHistBytes, s>>>(keys, Lk, B, idx);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fc

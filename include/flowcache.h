@@ -1,0 +1,205 @@
+/*
+ * libflowcache -- FlowCache's per-step hot path for NVIDIA B200 (sm_100a).
+ *
+ * Method: "Flow Caching for Autoregressive Video Generation" (paper notes on
+ * papernotes.org, ICLR 2026), section 方法详解 / 关键设计 (method details / key
+ * designs) 1-3.  Two parts:
+ *   - the chunkwise cache gate (key designs 1 and 2): a fused Euler update with
+ *     per-chunk relative-L1 reductions and the recursive accumulator f that
+ *     decides, per chunk, whether the next forward recomputes or reuses;
+ *   - the joint importance-redundancy KV-cache compression (key design 3):
+ *     importance, redundancy, pooled joint score, per-head top-B, and the
+ *     compaction of the kept K/V rows into the fixed B_budget buffer.
+ *
+ * Conventions shared by every call
+ *   - Every tensor pointer is a DEVICE pointer (cudaMalloc / torch CUDA
+ *     memory / managed memory) owned by the caller.  The library allocates
+ *     nothing and keeps no state between calls.  Host pointers are rejected
+ *     with FC_ERR_INVALID_ARG before anything is launched.
+ *   - Tensors are dense, row-major, with the stated layout, and their base
+ *     address is 16-byte aligned.  "[H][L][d]" means head-major.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
+ *     are asynchronous: they enqueue kernels and return.
+ *   - Arguments are validated on the host before any launch.  On any error
+ *     status nothing has been launched and no output was touched, except
+ *     FC_ERR_CUDA, which reports a failed launch (the message names it).
+ *     fc_last_error() returns a thread-local description of the last error.
+ *   - `ws` is caller-owned device scratch of at least the size returned by the
+ *     matching *_workspace_size() query.  Its contents are clobbered, except
+ *     where a call says otherwise.  Two calls that run at the same time on the
+ *     GPU must not share a workspace.
+ *   - Results are deterministic: the same inputs and sizes give bitwise the
+ *     same outputs (no floating-point atomics).
+ */
+#ifndef FLOWCACHE_H
+#define FLOWCACHE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FC_OK = 0,
+  FC_ERR_INVALID_ARG = 1, /* a null / host / misaligned pointer or a bad size     */
+  FC_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement         */
+  FC_ERR_WORKSPACE = 3,   /* ws is null or smaller than the *_workspace_size()     */
+  FC_ERR_CUDA = 4,        /* a CUDA call failed; see fc_last_error()               */
+  FC_ERR_TIMEOUT = 5      /* reserved: a bounded device-side wait gave up          */
+} fc_status;
+
+typedef enum { FC_F32 = 0, FC_BF16 = 1 } fc_dtype;
+
+/* Thread-local text of the last error reported on this thread ("" if none). */
+const char* fc_last_error(void);
+
+/* Library version, as major*10000 + minor*100 + patch. */
+int fc_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Chunkwise cache gate (key design 1: relative L1 distance; key design 2:  */
+/* the accumulator f)                                                       */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes for fc_chunk_l1_gate. */
+size_t fc_gate_workspace_size(int n_chunks, int64_t n_per_chunk);
+
+/*
+ * One denoising step of the chunkwise cache gate for every chunk.
+ *
+ * Key design 1 defines, for chunk i at step t, the relative L1 distance
+ *   L1_rel = ||X_{t-1} - X_t||_1 / ||X_t||_1 = ||v*dt||_1 / ||X_t||_1.
+ * Key design 2 keeps a per-chunk accumulator f: the first m steps of a chunk
+ * recompute (f = 0); afterwards, if f + L1_rel > eps the chunk recomputes
+ * and f resets to 0, otherwise f += L1_rel and the chunk reuses its cached
+ * activations.
+ *
+ * In one pass this call applies the Euler update X <- X + v*dt (float32:
+ * the product rounded once, then the sum rounded once; no fused
+ * multiply-add), forms ||v*dt||_1 and ||X_t||_1 (pre-update X) in float64,
+ * and runs the recurrence (in float32, compare strictly greater).
+ *
+ *   x          [n_chunks][n_per_chunk] float32, in/out: X_t in, X_{t-1} out
+ *   v          [n_chunks][n_per_chunk] float32, velocity applied this step
+ *   dt         [n_chunks] float32, signed step of each chunk
+ *   step       [n_chunks] int32, steps chunk c has taken since it started;
+ *              step < 0 marks an inactive chunk: x, f untouched, l1 = 0,
+ *              recompute = 0
+ *   m          forced-recompute steps (>= 0)
+ *   eps        threshold
+ *   f          [n_chunks] float32, in/out accumulator
+ *   l1_rel     [n_chunks] float32, out: L1_rel (+inf when ||X_t||_1 = 0 and
+ *              the update is not zero; 0 when both are zero)
+ *   recompute  [n_chunks] uint8, out: 1 = recompute at the chunk's next
+ *              forward, 0 = reuse
+ *   ws         fc_gate_workspace_size() bytes.  Its first
+ *              4*n_chunks bytes are completion counters that must be zero
+ *              before the first call (e.g. cudaMemsetAsync once); every call
+ *              leaves them zero again.
+ * Errors: n_chunks < 1, n_per_chunk < 0, m < 0, null/host/misaligned
+ * pointers -> FC_ERR_INVALID_ARG; small ws -> FC_ERR_WORKSPACE.
+ */
+fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
+                           const float* dt, const int32_t* step, int32_t m, float eps,
+                           float* f, float* l1_rel, uint8_t* recompute, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Joint importance-redundancy KV compression (key design 3)                */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes for fc_kv_importance. */
+size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d);
+
+/*
+ * Pre-pooling importance of every clean key, per head (key design 3):
+ *   Imp[h][j] = (1/Lq) * sum_q softmax_j(scale * q_q . k_j),
+ * the attention softmax of the current denoising queries over the Lk clean
+ * candidate keys, averaged over the queries.  Computed in two passes over
+ * Q K^T: the row log-sum-exp of every query, then the column sums of
+ * exp(s - lse).  Accumulation and softmax in float32.
+ *
+ *   q      [H][Lq][d] dtype, denoising queries
+ *   k      [H][Lk][d] dtype, clean keys
+ *   dtype  FC_BF16 (tensor-core path) or FC_F32 (CUDA-core path)
+ *   d      64 or 128
+ *   scale  logit scale; <= 0 selects 1/sqrt(d)
+ *   imp    [H][Lk] float32, out; each row sums to 1
+ *   ws     fc_importance_workspace_size() bytes (the per-query log-sum-exp)
+ * Errors: H, Lq, Lk < 1 or d not in {64, 128} -> FC_ERR_INVALID_ARG /
+ * FC_ERR_UNSUPPORTED; bad pointers -> FC_ERR_INVALID_ARG; small ws ->
+ * FC_ERR_WORKSPACE.
+ */
+fc_status fc_kv_importance(const void* q, const void* k, fc_dtype dtype, int H, int Lq, int Lk,
+                           int d, float scale, float* imp, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* Workspace bytes for fc_kv_redundancy. */
+size_t fc_redundancy_workspace_size(fc_dtype dtype, int H, int Lk, int d);
+
+/*
+ * Redundancy of every clean key, per head (key design 3):
+ *   Red[h][j] = softmax_j( (1/Lk) * sum_{i != j} khat_i . khat_j ),
+ * khat the l2-normalised keys (a zero key stays zero), i.e. the softmax of the
+ * column means of the cosine-similarity matrix with its diagonal zeroed.
+ * Evaluated with the exact identity sum_{i != j} khat_i.khat_j =
+ * khat_j.(sum_i khat_i) - ||khat_j||^2, so that K is streamed instead of the
+ * Lk x Lk matrix being formed.
+ *
+ *   k    [H][Lk][d] dtype
+ *   red  [H][Lk] float32, out; each row sums to 1
+ * Errors as for fc_kv_importance.
+ */
+fc_status fc_kv_redundancy(const void* k, fc_dtype dtype, int H, int Lk, int d, float* red,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Workspace bytes for fc_kv_score_topb. */
+size_t fc_score_topb_workspace_size(int H, int Lk, int B);
+
+/*
+ * Joint score and per-head top-B selection (key design 3):
+ *   Imp~ = 1D max filter of imp along the token axis (odd `pool_window`,
+ *          stride 1, output length Lk, taps outside [0, Lk) ignored),
+ *   Score[h][j] = lambda*Imp~[h][j] - (1-lambda)*Red[h][j], evaluated in
+ *          float32 as fl(fl(lambda*Imp~) - fl(fl(1-lambda)*Red)),
+ *   idx[h] = the B tokens with the largest Score; equal scores keep the lower
+ *          token index (-0 and +0 are equal); indices written ascending, which
+ *          keeps the temporal order of the kept tokens.
+ * B >= Lk keeps every token: idx[h][r] = r for r < Lk, -1 for r >= Lk.
+ *
+ *   imp, red     [H][Lk] float32 (outputs of the two calls above)
+ *   pool_window  odd, in [1, 511]
+ *   lambda       mixing weight (not clamped)
+ *   B            >= 1, tokens kept per head
+ *   score        [H][Lk] float32 out, or NULL to skip writing it
+ *   idx          [H][B] int32 out
+ * Errors: B < 1, pool_window even or out of range, bad pointers ->
+ * FC_ERR_INVALID_ARG;
+ * small ws -> FC_ERR_WORKSPACE.
+ */
+fc_status fc_kv_score_topb(const float* imp, const float* red, int H, int Lk, int pool_window,
+                           float lambda, int B, float* score, int32_t* idx, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/*
+ * Compaction of the kept rows into the fixed-budget buffer (key design 3: the
+ * compressed clean region B_budget of the fixed KV buffer):
+ *   k_out[h][r] = k[h][idx[h][r]],  v_out[h][r] = v[h][idx[h][r]],
+ * rows whose index is -1 are written as zeros.  Bitwise copy.
+ *
+ *   k, v          [H][Lk][d] dtype
+ *   idx           [H][B] int32, each entry in [0, Lk) or -1
+ *   k_out, v_out  [H][B][d] dtype, out; must not overlap k or v
+ * Errors: bad sizes or pointers, overlapping buffers -> FC_ERR_INVALID_ARG.
+ * An index outside [-1, Lk) is not read: the row is written as zeros.
+ */
+fc_status fc_kv_compact(const void* k, const void* v, fc_dtype dtype, int H, int Lk, int d,
+                        const int32_t* idx, int B, void* k_out, void* v_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLOWCACHE_H */

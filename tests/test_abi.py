@@ -1,0 +1,118 @@
+"""The C-ABI boundary on the host: the library loads, exports every call that
+include/*.h declares, and rejects bad arguments before launching anything.
+No test here needs a GPU (no compute call reaches a kernel)."""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import cache_gating_kv_b200 as fc
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+DECL = re.compile(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(fc_\w+)\s*\(", re.M)
+
+
+def _declared():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        names.update(DECL.findall(open(h).read()))
+    return sorted(names)
+
+
+def test_header_declares_the_calls():
+    names = _declared()
+    for n in ["fc_chunk_l1_gate", "fc_kv_importance", "fc_kv_redundancy", "fc_kv_score_topb",
+              "fc_kv_compact", "fc_last_error"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(fc.library_path)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_version_and_workspace_queries():
+    lib = fc.library()
+    assert lib.fc_version() >= 100
+    assert lib.fc_gate_workspace_size(4, 777600) > 0
+    assert lib.fc_gate_workspace_size(0, 10) == 0
+    assert lib.fc_importance_workspace_size(fc.FC_BF16, 24, 4096, 16384, 128) >= 24 * 4096 * 4
+    assert lib.fc_redundancy_workspace_size(fc.FC_BF16, 24, 16384, 128) > 0
+    assert lib.fc_redundancy_workspace_size(fc.FC_BF16, 24, 16384, 96) == 0
+    assert lib.fc_score_topb_workspace_size(24, 16384, 8192) >= 24 * 16384 * 4
+
+
+NULL = None
+
+
+def test_gate_rejects_bad_sizes_before_touching_memory():
+    lib = fc.library()
+    args = lambda n_c, N, m, ws_bytes: lib.fc_chunk_l1_gate(  # noqa: E731
+        NULL, NULL, n_c, N, NULL, NULL, m, 0.1, NULL, NULL, NULL, NULL, ws_bytes, NULL)
+    assert args(0, 10, 1, 1 << 20) == 1
+    assert args(70000, 10, 1, 1 << 30) == 1
+    assert args(2, -1, 1, 1 << 20) == 1
+    assert args(2, 10, -1, 1 << 20) == 1
+    assert args(2, 10, 1, 1 << 20) == 3  # ws is NULL -> workspace error
+    assert b"workspace" in lib.fc_last_error()
+
+
+def test_gate_rejects_null_tensor_with_message():
+    lib = fc.library()
+    ws = ctypes.create_string_buffer(1 << 20)
+    buf = ctypes.addressof(ws)
+    st = lib.fc_chunk_l1_gate(NULL, NULL, 2, 10, NULL, NULL, 1, 0.1, NULL, NULL, NULL, buf,
+                              1 << 20, NULL)
+    assert st == 1 and lib.fc_last_error() == b"x is NULL"
+
+
+def test_host_pointer_is_rejected():
+    """A host pointer never reaches a kernel: without a GPU the pointer query
+    fails (FC_ERR_CUDA); with one, host memory is FC_ERR_INVALID_ARG."""
+    lib = fc.library()
+    host = ctypes.create_string_buffer(1 << 16)
+    p = (ctypes.addressof(host) + 15) // 16 * 16
+    st = lib.fc_kv_compact(p, p, fc.FC_BF16, 1, 8, 128, p, 4, p + 4096, p + 8192, NULL)
+    assert st in (1, 4)
+    assert lib.fc_last_error() != b""
+
+
+def test_kv_calls_reject_bad_shapes():
+    lib = fc.library()
+    # d not in {64, 128}
+    assert lib.fc_kv_importance(NULL, NULL, fc.FC_BF16, 2, 8, 8, 96, 0.0, NULL, NULL, 0, NULL) == 2
+    assert lib.fc_kv_redundancy(NULL, fc.FC_BF16, 2, 8, 32, NULL, NULL, 0, NULL) == 2
+    # empty sizes
+    assert lib.fc_kv_importance(NULL, NULL, fc.FC_BF16, 0, 8, 8, 64, 0.0, NULL, NULL, 0, NULL) == 1
+    assert lib.fc_kv_importance(NULL, NULL, fc.FC_BF16, 2, 0, 8, 64, 0.0, NULL, NULL, 0, NULL) == 1
+    # unknown dtype
+    assert lib.fc_kv_redundancy(NULL, 7, 2, 8, 64, NULL, NULL, 0, NULL) == 1
+    # workspace too small
+    assert lib.fc_kv_importance(NULL, NULL, fc.FC_BF16, 2, 8, 8, 64, 0.0, NULL, NULL, 4, NULL) == 3
+    # score/top-B: B < 1, even or too wide pool window
+    assert lib.fc_kv_score_topb(NULL, NULL, 2, 8, 7, 0.5, 0, NULL, NULL, NULL, 1 << 20, NULL) == 1
+    assert lib.fc_kv_score_topb(NULL, NULL, 2, 8, 6, 0.5, 4, NULL, NULL, NULL, 1 << 20, NULL) == 1
+    assert lib.fc_kv_score_topb(NULL, NULL, 2, 8, 513, 0.5, 4, NULL, NULL, NULL, 1 << 20,
+                                NULL) == 1
+    assert lib.fc_kv_compact(NULL, NULL, fc.FC_BF16, 2, 8, 64, NULL, 0, NULL, NULL, NULL) == 1
+    assert lib.fc_kv_compact(NULL, NULL, fc.FC_BF16, 2, 8, 64, NULL, 4, NULL, NULL, NULL) == 1
+
+
+def test_binding_fails_loudly_without_cuda_tensors():
+    import torch
+    x = torch.zeros(2, 8)
+    with pytest.raises(fc.FlowCacheError):
+        fc.fc_kv_redundancy(x.view(1, 2, 8), torch.zeros(1, 2), torch.zeros(256, dtype=torch.uint8))
+
+
+def test_product_package_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "cache_gating_kv_b200")
+    for path in glob.glob(os.path.join(pkg, "**", "*.py"), recursive=True) + \
+            glob.glob(os.path.join(pkg, "csrc", "*")):
+        src = open(path, errors="replace").read()
+        assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), path
+        assert "flowcache_oracle" not in src, path

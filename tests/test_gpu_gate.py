@@ -1,0 +1,131 @@
+"""GPU parity of fc_chunk_l1_gate against the CPU oracle.
+
+The Euler update must match bitwise; L1_rel to 1e-6 relative (both sides sum
+in float64); the recompute mask and f exactly, except for chunks whose
+oracle margin |f + L1 - eps| is below 1e-5 (the margin waiver)."""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import cache_gating_kv_b200 as fc
+from cache_gating_kv_b200 import workloads as W
+from oracle import flowcache_oracle as O
+from tests.gpu_util import gate_gpu
+
+pytestmark = pytest.mark.gpu
+MARGIN = 1e-5
+
+
+def _compare(out_gpu, out_ref, f_prev, step, m, eps):
+    xg, fg, lg, mg = out_gpu
+    xr, fr, lr, mr = out_ref
+    np.testing.assert_array_equal(xg.view(np.uint32), xr.view(np.uint32))
+    np.testing.assert_allclose(lg, lr, rtol=1e-6, atol=0)
+    for c in range(len(mr)):
+        margin = abs(float(np.float32(f_prev[c] + lr[c])) - eps) if step[c] >= m else 1.0
+        if margin < MARGIN:
+            continue
+        assert mg[c] == mr[c], f"chunk {c}: mask {mg[c]} vs {mr[c]}"
+        assert fg[c] == pytest.approx(fr[c], rel=1e-6, abs=0), f"chunk {c}"
+
+
+def test_gate_hand_trace_on_gpu(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "gate_trace_constant.json")))
+    N = g["N"]
+    f = np.zeros(1, np.float32)
+    ws = fc.workspace(fc.fc_gate_workspace_size(1, N))
+    for t in range(g["steps"]):
+        x = np.full((1, N), g["x"], np.float32)
+        v = np.full((1, N), g["v"], np.float32)
+        xn, f, l1, mask = gate_gpu(x, v, [g["dt"]], [t], g["m"], g["eps"], f, ws=ws)
+        assert l1[0] == np.float32(g["l1"][t])
+        assert mask[0] == g["mask"][t]
+        assert f[0] == np.float32(g["f"][t])
+        assert np.all(xn == np.float32(g["x_next"]))
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "bf16_layer", "bf16_large_head", "full_step_sweep"])
+def test_gate_step_parity_on_workloads(name):
+    cfg = W.GATE_CONFIGS[name]
+    x = W.gate_initial(cfg, seed=0)
+    v = W.gate_velocity(cfg, seed=0)
+    rng = np.random.default_rng(1)
+    ws = fc.workspace(fc.fc_gate_workspace_size(cfg.n_chunks, cfg.N))
+    for eps in cfg.eps:
+        for gstep in (0, cfg.m, cfg.T // 2 + cfg.stagger * (cfg.n_chunks - 1) // 2):
+            step = W.gate_step_counters(cfg, gstep)
+            dt = W.gate_dt(cfg, step)
+            f = (rng.random(cfg.n_chunks) * eps).astype(np.float32)
+            ref = O.gate_step(x, v, dt, step, cfg.m, eps, f)
+            got = gate_gpu(x, v, dt, step, cfg.m, eps, f, ws=ws)
+            _compare(got, ref, f, step, cfg.m, eps)
+
+
+def test_gate_trajectory_with_reuse_feedback():
+    """tiny workload over all T steps: a recompute draws a fresh velocity, a
+    reuse re-applies the cached one; GPU and oracle advance side by side."""
+    cfg = W.GATE_CONFIGS["tiny_fp32"]
+    eps = cfg.eps[0]
+    x_r = x_g = W.gate_initial(cfg, 0)
+    f_r = f_g = np.zeros(cfg.n_chunks, np.float32)
+    v_cache = W.gate_velocity(cfg, 0, draw=0)
+    mask = np.ones(cfg.n_chunks, np.uint8)
+    for t in range(cfg.T):
+        fresh = W.gate_velocity(cfg, 0, draw=t)
+        v = np.where(mask[:, None] == 1, fresh, v_cache).astype(np.float32)
+        v_cache = v
+        step = np.full(cfg.n_chunks, t, np.int32)
+        dt = W.gate_dt(cfg, step)
+        ref = O.gate_step(x_r, v, dt, step, cfg.m, eps, f_r)
+        got = gate_gpu(x_g, v, dt, step, cfg.m, eps, f_g)
+        _compare(got, ref, f_r, step, cfg.m, eps)
+        x_r, f_r, _, mask = ref
+        x_g, f_g = got[0], got[1]
+        np.testing.assert_array_equal(got[3], mask)
+
+
+@pytest.mark.parametrize("n_c,N", [(1, 1), (3, 5), (5, 1001), (2, 3), (7, 4099), (1, 0)])
+def test_gate_ragged_and_misaligned_chunks(n_c, N):
+    rng = np.random.default_rng(N + n_c)
+    x = rng.standard_normal((n_c, N)).astype(np.float32)
+    v = rng.standard_normal((n_c, N)).astype(np.float32)
+    dt = rng.uniform(-0.1, 0.1, n_c).astype(np.float32)
+    step = np.arange(n_c, dtype=np.int32)
+    f = (rng.random(n_c) * 0.1).astype(np.float32)
+    ref = O.gate_step(x, v, dt, step, 1, 0.3, f)
+    got = gate_gpu(x, v, dt, step, 1, 0.3, f)
+    _compare(got, ref, f, step, 1, 0.3)
+
+
+def test_gate_inactive_zero_norm_and_forced_steps():
+    N = 4096
+    x = np.stack([np.ones(N), np.zeros(N), np.zeros(N), np.ones(N), np.ones(N)]).astype(np.float32)
+    v = np.stack([np.ones(N), np.ones(N), np.zeros(N), np.ones(N), np.ones(N)]).astype(np.float32)
+    dt = np.float32([0.5, 0.5, 0.5, 0.5, 1e-4])
+    step = np.int32([-1, 7, 7, 7, 2])
+    f = np.float32([0.5, 0.0, 0.0, 0.25, 0.4])
+    ref = O.gate_step(x, v, dt, step, 3, 100.0, f)
+    got = gate_gpu(x, v, dt, step, 3, 100.0, f)
+    _compare(got, ref, f, step, 3, 100.0)
+    assert np.isinf(got[2][1]) and got[3][1] == 1
+    assert got[2][0] == 0 and got[3][0] == 0 and got[1][0] == np.float32(0.5)
+    assert got[3][4] == 1 and got[1][4] == 0  # step 2 < m = 3: forced
+
+
+def test_gate_deterministic_and_counters_reset():
+    cfg = W.GATE_CONFIGS["bf16_layer"]
+    x = W.gate_initial(cfg, 3)
+    v = W.gate_velocity(cfg, 3)
+    step = np.full(cfg.n_chunks, 10, np.int32)
+    dt = W.gate_dt(cfg, step)
+    f = np.zeros(cfg.n_chunks, np.float32)
+    ws = fc.workspace(fc.fc_gate_workspace_size(cfg.n_chunks, cfg.N))
+    a = gate_gpu(x, v, dt, step, cfg.m, 0.01, f, ws=ws)
+    b = gate_gpu(x, v, dt, step, cfg.m, 0.01, f, ws=ws)
+    for u, w in zip(a, b):
+        np.testing.assert_array_equal(u, w)
+    assert int(ws[: 4 * cfg.n_chunks].sum()) == 0  # completion counters back at zero
