@@ -107,7 +107,7 @@ class Clocks:
         mx = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)
         loaded = [m for m in mhz if mx and m > 0.5 * mx] or mhz
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i]})
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
         return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
                 "reasons": reasons, "samples": len(rows)}
 

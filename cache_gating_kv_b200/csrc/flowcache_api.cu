@@ -108,8 +108,10 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
   if (m < 0) return fail(FC_ERR_INVALID_ARG, "m must be >= 0");
   if (ws == nullptr || ws_bytes < fc::gate_ws_bytes(n_chunks))
     return fail(FC_ERR_WORKSPACE, "gate workspace needs %zu bytes", fc::gate_ws_bytes(n_chunks));
-  FC_CHECK_PTR(x);
-  FC_CHECK_PTR(v);
+  if (n_per_chunk > 0) {  // empty chunks touch no latent memory
+    FC_CHECK_PTR(x);
+    FC_CHECK_PTR(v);
+  }
   FC_CHECK_PTR(dt);
   FC_CHECK_PTR(step);
   FC_CHECK_PTR(f);

@@ -189,11 +189,9 @@ cudaError_t run(const T* q, const T* k, int H, int Lq, int Lk, float scale, floa
 }
 }  // namespace
 
-size_t importance_ws_bytes(int H, int Lq) { return align_up((size_t)H * Lq * sizeof(float), 256); }
-
 cudaError_t launch_importance_simt(const void* q, const void* k, bool bf16, int H, int Lq, int Lk,
                                    int d, float scale, float* imp, void* ws, cudaStream_t s) {
-  float* lse2 = static_cast<float*>(ws);
+  float* lse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);  // after the error word
   if (bf16) {
     const auto* qb = static_cast<const __nv_bfloat16*>(q);
     const auto* kb = static_cast<const __nv_bfloat16*>(k);

@@ -98,6 +98,8 @@ size_t fc_gate_workspace_size(int n_chunks, int64_t n_per_chunk);
  *              4*n_chunks bytes are completion counters that must be zero
  *              before the first call (e.g. cudaMemsetAsync once); every call
  *              leaves them zero again.
+ * x and v may be NULL when n_per_chunk == 0 (then L1_rel = 0 for every
+ * active chunk).
  * Errors: n_chunks < 1, n_per_chunk < 0, m < 0, null/host/misaligned
  * pointers -> FC_ERR_INVALID_ARG; small ws -> FC_ERR_WORKSPACE.
  */
@@ -127,7 +129,11 @@ size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d
  *   d      64 or 128
  *   scale  logit scale; <= 0 selects 1/sqrt(d)
  *   imp    [H][Lk] float32, out; each row sums to 1
- *   ws     fc_importance_workspace_size() bytes (the per-query log-sum-exp)
+ *   ws     fc_importance_workspace_size() bytes: bytes 0..3 are an error
+ *          word that the tensor-core path sets to nonzero if one of its
+ *          bounded device-side waits gave up (the call never clears it; zero
+ *          it once, read it after synchronizing); the per-query log-sum-exp
+ *          follows from byte 256
  * Errors: H, Lq, Lk < 1 or d not in {64, 128} -> FC_ERR_INVALID_ARG /
  * FC_ERR_UNSUPPORTED; bad pointers -> FC_ERR_INVALID_ARG; small ws ->
  * FC_ERR_WORKSPACE.

@@ -40,6 +40,7 @@ def importance_gpu(q, k, scale=0.0):
     ws = fc.workspace(fc.fc_importance_workspace_size(code, H, Lq, Lk, d))
     fc.fc_kv_importance(q.to(DEV), k.to(DEV), imp, ws, scale=scale)
     torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0, "a bounded device wait gave up"
     return imp.cpu().numpy()
 
 
