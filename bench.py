@@ -182,6 +182,23 @@ class Step:
         self.d["f"].zero_()
 
 
+def reduce_max(values, world, device):
+    """Element-wise max over ranks of a few host floats (identity at world 1)."""
+    if world <= 1:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return [float(v) for v in t.cpu()]
+
+
+def shard_heads(H, rank, world):
+    """Contiguous head range [lo, hi) of `rank` when one layer's heads are split
+    over `world` GPUs (every head is independent: no exchange is needed)."""
+    per, extra = divmod(H, world)
+    lo = rank * per + min(rank, extra)
+    return lo, lo + per + (1 if rank < extra else 0)
+
+
 def _bytes_gate(gc):
     return 12 * gc.n_chunks * gc.N
 
@@ -232,13 +249,10 @@ def native(a, rank, world, local_rank):
     if not a.no_e2e:
         e2e = _e2e(step, stream, flush, a, dev)
 
-    t_max = ms_step
-    if world > 1:
-        t = torch.tensor([ms_step] + ([e2e["ms"]] if e2e else []), device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_max = float(t[0])
-        if e2e:
-            e2e["ms"] = float(t[1])
+    maxed = reduce_max([ms_step] + ([e2e["ms"]] if e2e else []), world, dev)
+    t_max = maxed[0]
+    if e2e:
+        e2e["ms"] = maxed[1]
     H, Lq, Lk, d = kv_cfg.H, kv_cfg.Lq, kv_cfg.Lk, kv_cfg.d
     value = world * Lk / (t_max * 1e-3)  # tokens/s per head over all ranks
     hbm, tf_burst, tf_sus, src = _peaks()
