@@ -23,6 +23,7 @@ __all__ = [
     "library_path",
     "fc_version",
     "fc_chunk_l1_gate",
+    "fc_chunk_l1_gate_noalloc",
     "fc_kv_importance",
     "fc_kv_redundancy",
     "fc_kv_score_topb",
@@ -59,6 +60,8 @@ def _declare(lib):
         "fc_gate_workspace_size": (c_sz, [c_int, c_i64]),
         "fc_chunk_l1_gate": (c_int, [c_p, c_p, c_int, c_i64, c_p, c_p, ctypes.c_int32, c_f, c_p,
                                      c_p, c_p, c_p, c_sz, c_p]),
+        "fc_chunk_l1_gate_noalloc": (c_int, [c_p, c_p, c_int, c_i64, c_p, c_p, ctypes.c_int32,
+                                             c_f, c_p, c_p, c_p, c_p]),
         "fc_importance_workspace_size": (c_sz, [c_int, c_int, c_int, c_int, c_int]),
         "fc_kv_importance": (c_int, [c_p, c_p, c_int, c_int, c_int, c_int, c_int, c_f, c_p, c_p,
                                      c_sz, c_p]),
@@ -157,6 +160,18 @@ def fc_chunk_l1_gate(x, v, dt, step, m, eps, f, l1_rel, recompute, ws, stream=No
                                      _p(f), _p(l1_rel), _p(recompute), _p(ws), ws.numel(),
                                      _s(stream))
     _check("fc_chunk_l1_gate", st)
+
+
+def fc_chunk_l1_gate_noalloc(x, v, dt, step, m, eps, f, l1_rel, recompute, stream=None):
+    """The gate step without a workspace, for callers that cannot allocate
+    device memory while they run it (the library keeps a fixed static scratch
+    array instead).  At most 32 chunks per call; calls must not overlap on the
+    GPU; the first call on a device should precede any stream capture."""
+    n_c, N = x.shape
+    st = library().fc_chunk_l1_gate_noalloc(_p(x), _p(v), n_c, N, _p(dt), _p(step), int(m),
+                                             float(eps), _p(f), _p(l1_rel), _p(recompute),
+                                             _s(stream))
+    _check("fc_chunk_l1_gate_noalloc", st)
 
 
 def fc_kv_importance(q, k, imp, ws, scale=0.0, stream=None):

@@ -14,6 +14,13 @@ cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t n_per_ch
                         const float* dt, const int32_t* step, int m, float eps, float* f,
                         float* l1, uint8_t* mask, void* ws, cudaStream_t s);
 
+// Same kernel with its scratch in a static device array (no allocation, at
+// most gate_noalloc_max_chunks() chunks; calls must not overlap on the GPU).
+int gate_noalloc_max_chunks();
+cudaError_t launch_gate_noalloc(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
+                                const float* dt, const int32_t* step, int m, float eps, float* f,
+                                float* l1, uint8_t* mask, cudaStream_t s);
+
 // ---- importance --------------------------------------------------------------
 size_t importance_ws_bytes(int H, int Lq);
 // bf16 tensor-core path (tcgen05 + TMEM + TMA)

@@ -123,6 +123,31 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
                   "fc_chunk_l1_gate");
 }
 
+fc_status fc_chunk_l1_gate_noalloc(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
+                                   const float* dt, const int32_t* step, int32_t m, float eps,
+                                   float* f, float* l1_rel, uint8_t* recompute, void* stream) {
+  const int max_chunks = fc::gate_noalloc_max_chunks();
+  if (n_chunks < 1 || n_chunks > max_chunks)
+    return fail(FC_ERR_INVALID_ARG,
+                "fc_chunk_l1_gate_noalloc serves 1 to %d chunks per call (got %d); use "
+                "fc_chunk_l1_gate with a workspace for more",
+                max_chunks, n_chunks);
+  if (n_per_chunk < 0) return fail(FC_ERR_INVALID_ARG, "n_per_chunk must be >= 0");
+  if (m < 0) return fail(FC_ERR_INVALID_ARG, "m must be >= 0");
+  if (n_per_chunk > 0) {
+    FC_CHECK_PTR(x);
+    FC_CHECK_PTR(v);
+  }
+  FC_CHECK_PTR(dt);
+  FC_CHECK_PTR(step);
+  FC_CHECK_PTR(f);
+  FC_CHECK_PTR(l1_rel);
+  FC_CHECK_PTR(recompute);
+  return launched(fc::launch_gate_noalloc(x, v, n_chunks, n_per_chunk, dt, step, m, eps, f,
+                                          l1_rel, recompute, static_cast<cudaStream_t>(stream)),
+                  "fc_chunk_l1_gate_noalloc");
+}
+
 size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d) {
   (void)dtype;
   (void)Lk;

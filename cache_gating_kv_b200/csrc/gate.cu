@@ -196,4 +196,56 @@ cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t N, const
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// Allocation-free variant of the gate.
+//
+// Some callers cannot allocate device memory when they run the gate: a host
+// runtime that gives its plugins only their input and output buffers and
+// forbids cudaMalloc while work is being enqueued (an allocation may
+// synchronize the device, or fail under a fixed memory budget), or code that
+// has nowhere to keep a workspace alive between denoising steps.  For them
+// the gate's scratch (completion counters and per-block partial sums) lives in
+// one file-scope device array of a fixed size: every GPU that loads this
+// library holds it until the process exits.  It serves at most
+// kGateNoAllocMaxChunks chunks per call.  Every call shares the array, so
+// calls that overlap on the GPU (other streams, other host threads) race;
+// they must be ordered.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int kGateNoAllocMaxChunks = 32;
+constexpr size_t kGateNoAllocBytes =
+    256 + (size_t)kGateNoAllocMaxChunks * kGateMaxBlocksPerChunk * sizeof(double2);  // 512.25 KiB
+
+static __device__ __align__(256) unsigned char g_gate_scratch[kGateNoAllocBytes];
+
+// Device address of g_gate_scratch per device ordinal, filled on the first
+// call made with that device current.  In host code the array's name is only
+// a host-side stand-in, so the address must come from cudaGetSymbolAddress.
+void* g_gate_scratch_addr[128] = {nullptr};
+}  // namespace
+
+int gate_noalloc_max_chunks() { return kGateNoAllocMaxChunks; }
+
+cudaError_t launch_gate_noalloc(float* x, const float* v, int n_chunks, int64_t N,
+                                const float* dt, const int32_t* step, int m, float eps, float* f,
+                                float* l1, uint8_t* mask, cudaStream_t s) {
+  if (n_chunks < 1 || n_chunks > kGateNoAllocMaxChunks) return cudaErrorInvalidValue;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  if (g_gate_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_gate_scratch);
+    if (e != cudaSuccess) return e;
+    g_gate_scratch_addr[dev] = p;
+  }
+  void* ws = g_gate_scratch_addr[dev];
+  // The completion counters must start at zero; the array keeps whatever the
+  // previous call left, so clear them on the caller's stream first.
+  e = cudaMemsetAsync(ws, 0, (size_t)n_chunks * sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+  return launch_gate(x, v, n_chunks, N, dt, step, m, eps, f, l1, mask, ws, s);
+}
+
 }  // namespace fc

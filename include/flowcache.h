@@ -108,6 +108,34 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
                            float* f, float* l1_rel, uint8_t* recompute, void* ws,
                            size_t ws_bytes, void* stream);
 
+/*
+ * Allocation-free variant of fc_chunk_l1_gate.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory when
+ * they run the gate -- for example a host runtime that hands its plugins only
+ * input and output buffers and forbids cudaMalloc while work is enqueued (an
+ * allocation can synchronize the device or fail under a fixed memory budget),
+ * or code with nowhere to keep a workspace alive between steps.
+ *
+ * Same arguments, results and errors as fc_chunk_l1_gate, without ws/ws_bytes.
+ * The scratch (completion counters and per-block partial sums) is one static
+ * device array of about 512 KiB inside the library, which every GPU that loads
+ * the library holds until the process exits.  Limits and behaviour:
+ *   - n_chunks must be in [1, 32]; larger counts return FC_ERR_INVALID_ARG
+ *     before anything is launched (use fc_chunk_l1_gate with a workspace).
+ *   - The call allocates nothing: no cudaMalloc, cudaFree or allocating
+ *     library routine.  It clears the counters it needs with an asynchronous
+ *     memset on `stream`, then launches the gate kernel.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture.
+ *   - Every call shares the one array: calls whose work overlaps on the GPU
+ *     (other streams, other host threads) race and give wrong results; order
+ *     them on one stream or with events.
+ */
+fc_status fc_chunk_l1_gate_noalloc(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
+                                   const float* dt, const int32_t* step, int32_t m, float eps,
+                                   float* f, float* l1_rel, uint8_t* recompute, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Joint importance-redundancy KV compression (key design 3)                */
 /* ------------------------------------------------------------------------ */
