@@ -5,6 +5,7 @@
 #include <cstring>
 
 #include "../../include/flowcache.h"
+#include "../../include/flowcache_selftest.h"
 #include "fc_common.cuh"
 #include "fc_kernels.h"
 
@@ -243,6 +244,16 @@ fc_status fc_kv_compact(const void* k, const void* v, fc_dtype dtype, int H, int
   return launched(fc::launch_compact(k, v, (int)elem_bytes(dtype), H, Lk, d, idx, B, k_out, v_out,
                                      static_cast<cudaStream_t>(stream)),
                   "fc_kv_compact");
+}
+
+fc_status fc_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n, void* stream) {
+  if (n < 0 || n % 2 != 0) return fail(FC_ERR_INVALID_ARG, "n must be even and >= 0");
+  if (n == 0) return ok();
+  FC_CHECK_PTR(x);
+  FC_CHECK_PTR(y_mufu);
+  FC_CHECK_PTR(y_poly);
+  return launched(fc::launch_exp2_selftest(x, y_mufu, y_poly, n, static_cast<cudaStream_t>(stream)),
+                  "fc_selftest_exp2");
 }
 
 }  // extern "C"

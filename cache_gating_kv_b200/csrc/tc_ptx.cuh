@@ -151,10 +151,68 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // ---- arithmetic -----------------------------------------------------------------
+// 2^x on the special-function unit (MUFU.EX2, ~2 ulp; flushes subnormals).
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Packed float32 pairs (sm_100 f32x2 arithmetic: two lanes per instruction).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)),
+        "l"(reinterpret_cast<const uint64_t&>(c)));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(reinterpret_cast<uint64_t&>(d))
+      : "l"(reinterpret_cast<const uint64_t&>(a)), "l"(reinterpret_cast<const uint64_t&>(b)));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair, on the FMA pipes instead of the special-function unit, so
+// that part of a tile's exponentials can run beside the MUFU ones.  Method:
+// Cody-Waite style range reduction x = n + f with n = round(x) (the
+// 1.5*2^23 rounding constant) and f in [-1/2, 1/2], a degree-5 polynomial for
+// 2^f whose coefficients we fitted (iteratively reweighted least squares for
+// relative error on Chebyshev nodes; cache_gating_kv_b200/csrc/gen_exp2_poly.py),
+// then n is added to the exponent field.  Max relative error 2.4e-7 for
+// x >= -125; inputs below -125 (including -inf) are clamped there, giving
+// about 2^-125 instead of 0.  With kClampHigh, inputs above 64 are clamped to
+// 64 (callers that must see overflow as a large value); without it the caller
+// guarantees x <= 126.
+template <bool kClampHigh>
+__device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  if (kClampHigh) {
+    x.x = fminf(x.x, 64.0f);
+    x.y = fminf(x.y, 64.0f);
+  }
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 j = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = fadd2(x, make_float2(-j.x, -j.y));
+  float2 p = make_float2(1.3278164e-03f, 1.3278164e-03f);
+  p = ffma2(p, f, make_float2(9.6755559e-03f, 9.6755559e-03f));
+  p = ffma2(p, f, make_float2(5.5507079e-02f, 5.5507079e-02f));
+  p = ffma2(p, f, make_float2(2.4022119e-01f, 2.4022119e-01f));
+  p = ffma2(p, f, make_float2(6.9314694e-01f, 6.9314694e-01f));
+  p = ffma2(p, f, make_float2(1.0000001e+00f, 1.0000001e+00f));
+  // the low bits of t hold n (two's complement); n << 23 lands in the exponent
+  const uint32_t ex = (__float_as_uint(t.x) << 23) + __float_as_uint(p.x);
+  const uint32_t ey = (__float_as_uint(t.y) << 23) + __float_as_uint(p.y);
+  return make_float2(__uint_as_float(ex), __uint_as_float(ey));
 }
 
 }  // namespace tc
