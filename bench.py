@@ -35,8 +35,16 @@ sys.path.insert(0, ROOT)
 METRIC = "clean KV tokens scored+selected/s per head; L1-gate GB/s; % of roofline"
 UNIT = "tokens/s/head"
 FLUSH_BYTES = 256 << 20  # > 126 MB L2
+
+
+def flush_l2(buf, sink):
+    """Evict every cached line: write a buffer larger than L2, then read it
+    back so the dirty lines are written back now and the next timed kernel
+    starts with a clean L2 (no write-back traffic of ours lands on it)."""
+    buf.zero_()
+    torch.sum(buf.view(torch.float32), dim=0, out=sink)
 # Kernel launches per call, as implemented in cache_gating_kv_b200/csrc.
-LAUNCHES = {"gate": 1, "importance": 2, "redundancy": 3, "score_topb": 2, "compact": 1}
+LAUNCHES = {"gate": 1, "importance": 2, "redundancy": 1, "score_topb": 2, "compact": 1}
 
 
 def _args():
@@ -212,6 +220,7 @@ def native(a, rank, world, local_rank):
     step = Step(kv_cfg, gate_cfg, seed=rank, dev=dev)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    sink = torch.empty((), dtype=torch.float32, device=dev)
     names = ["gate", "importance", "redundancy", "score_topb", "compact"]
 
     def barrier():
@@ -220,7 +229,7 @@ def native(a, rank, world, local_rank):
 
     with torch.cuda.stream(stream):
         for _ in range(a.warmup):
-            flush.zero_()
+            flush_l2(flush, sink)
             step.run(stream)
         stream.synchronize()
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(a.steps)]
@@ -229,7 +238,7 @@ def native(a, rank, world, local_rank):
         torch.cuda.synchronize()
         clocks.start()
         for i in range(a.steps):
-            flush.zero_()  # L2 flush between steps, outside the timed events
+            flush_l2(flush, sink)  # between steps, outside the timed events
             step.run(stream, evs[i])
         stream.synchronize()
         torch.cuda.synchronize()
@@ -247,7 +256,7 @@ def native(a, rank, world, local_rank):
     # end to end through the public API with host buffers (pinned), every step
     e2e = None
     if not a.no_e2e:
-        e2e = _e2e(step, stream, flush, a, dev)
+        e2e = _e2e(step, stream, flush, sink, a, dev)
 
     maxed = reduce_max([ms_step] + ([e2e["ms"]] if e2e else []), world, dev)
     t_max = maxed[0]
@@ -273,7 +282,8 @@ def native(a, rank, world, local_rank):
                                f"lambda={step.lam} pool={kv_cfg.pool}; gate {gate_cfg.n_chunks}x"
                                f"{gate_cfg.N} fp32 m={gate_cfg.m} eps={step.eps}",
                    "per_rank": "one independent layer per GPU",
-                   "l2": "flushed between steps (256 MiB write, outside the timed events)"},
+                   "l2": "flushed between steps (256 MiB write + read-back, outside the timed "
+                         "events)"},
         "roofline": {"bound": "tensor", "kernel": "fc_kv_importance (2 passes)",
                      "achieved": imp_tf, "peak": tf_burst, "unit": "TFLOP/s",
                      "frac": imp_tf / tf_burst, "peak_source": f"{src} bf16 burst",
@@ -292,7 +302,7 @@ def native(a, rank, world, local_rank):
     return out
 
 
-def _e2e(step, stream, flush, a, dev):
+def _e2e(step, stream, flush, sink, a, dev):
     """Same step with pinned host inputs copied in and the results read back,
     inside the timed region, every step."""
     host_in = {n: t.pin_memory() for n, t in step.host.items()}
@@ -305,7 +315,7 @@ def _e2e(step, stream, flush, a, dev):
     times = []
     with torch.cuda.stream(stream):
         for i in range(a.warmup + a.steps):
-            flush.zero_()
+            flush_l2(flush, sink)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             for n, t in host_in.items():

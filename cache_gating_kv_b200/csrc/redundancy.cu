@@ -6,31 +6,40 @@
 //
 // The L_k x L_k matrix is never formed.  With s = sum_i khat_i,
 //   sum_{i != j} khat_i . khat_j = khat_j . s - ||khat_j||^2      (exact)
-// so the logits r_j need one reduction pass over K and one dot pass.  r_j lies
-// in [-1, 1], hence exp(r_j) cannot overflow and the softmax needs no max.
+// so the logits r_j need one reduction over K and one dot pass.  r_j lies in
+// [-1, 1], hence exp(r_j) cannot overflow and the softmax needs no max.
 //
-//   pass A  grid (blocks_per_head, H): normalise rows, per-block partial s
-//   pass B  same grid: fixed-order sum of the partials -> s, then for every
-//           row r_j and e_j = exp(r_j) (written to red), per-block partial sum
-//   pass C  grid over H x L_k: fixed-order sum of the partials -> Z, red = e/Z
-// Each 16-byte lane vector holds 8 bf16 or 4 fp32 elements; a row of d
-// elements is spread over d*elem/16 lanes of a warp, so loads are coalesced
-// 16-byte vectors and every reduction runs in a fixed order (deterministic).
+// One kernel, one thread-block cluster per head (8 or 16 CTAs, each owning a
+// contiguous slice of the head's rows):
+//   1. every CTA sums khat over its rows; the partial d-vectors are exchanged
+//      through distributed shared memory and every CTA adds them in rank order
+//      (identical s everywhere, deterministic);
+//   2. every CTA re-reads its rows (now L2-resident), forms r_j and
+//      e_j = exp(r_j), writes e_j, and the per-CTA sums of e_j are exchanged
+//      the same way;
+//   3. every CTA scales its rows by 1/sum_j e_j.
+// The cluster barriers are hardware barriers (no spin loops).  Each 16-byte
+// lane vector holds 8 bf16 or 4 fp32 elements; a row is d*elem/16 lanes of a
+// warp, and every lane keeps four rows' loads in flight.
+#include <cooperative_groups.h>
+
 #include "fc_common.cuh"
 #include "fc_kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace fc {
 
 namespace {
 constexpr int kRedThreads = 256;
 constexpr int kRedWarps = kRedThreads / 32;
-constexpr int kRedMaxBlocksPerHead = 512;
+constexpr int kRedUnroll = 4;
 
 template <typename T, int D>
 struct RowLayout {
-  static constexpr int EPL = Vec16<T>::N;        // elements per lane
-  static constexpr int LPR = D / EPL;            // lanes per row
-  static constexpr int RPW = 32 / LPR;           // rows per warp step
+  static constexpr int EPL = Vec16<T>::N;  // elements per lane
+  static constexpr int LPR = D / EPL;      // lanes per row
+  static constexpr int RPW = 32 / LPR;     // rows per warp step
   static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "row layout");
 };
 
@@ -43,52 +52,64 @@ __device__ __forceinline__ float row_sum(float v) {
   return v;
 }
 
-__device__ __forceinline__ void block_rows(int Lk, int bph, int b, int& lo, int& hi) {
-  const int per = (int)ceil_div(Lk, bph);
-  lo = min(Lk, per * b);
-  hi = min(Lk, lo + per);
+template <typename T, int D>
+__device__ __forceinline__ void load_rows(const T* kh, int r0, int hi, int sub, int cl,
+                                          float (&e)[kRedUnroll][RowLayout<T, D>::EPL]) {
+  using L = RowLayout<T, D>;
+  uint4 u[kRedUnroll];
+#pragma unroll
+  for (int i = 0; i < kRedUnroll; ++i) {
+    const int r = r0 + i * L::RPW + sub;
+    u[i] = r < hi ? ld_nc_v4(kh + (size_t)r * D + cl * L::EPL) : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int i = 0; i < kRedUnroll; ++i) Vec16<T>::to_float(u[i], e[i]);
 }
 
-// Pass A: partial_s[h][b][:] = sum over this block's rows of khat.
 template <typename T, int D>
 __global__ void __launch_bounds__(kRedThreads)
-    red_sum_kernel(const T* __restrict__ k, int Lk, int bph, float* __restrict__ partial_s) {
+    red_cluster_kernel(const T* __restrict__ k, int Lk, float* __restrict__ red) {
   using L = RowLayout<T, D>;
-  const int h = blockIdx.y, b = blockIdx.x;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int nrank = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / L::LPR, cl = lane % L::LPR;
-  int lo, hi;
-  block_rows(Lk, bph, b, lo, hi);
+  const int per = (int)ceil_div(Lk, nrank);
+  const int lo = min(Lk, rank * per), hi = min(Lk, lo + per);
   const T* kh = k + (size_t)h * Lk * D;
+  constexpr int kRowsPerIter = kRedWarps * L::RPW * kRedUnroll;
 
+  __shared__ float s_acc[kRedWarps][D];
+  __shared__ float s_part[D];  // this CTA's sum of khat (read by the whole cluster)
+  __shared__ float s_vec[D];   // the head's s
+  __shared__ double s_esum[kRedWarps];
+  __shared__ double s_epart;   // this CTA's sum of e (read by the whole cluster)
+  __shared__ float s_inv;
+
+  // ---- 1. sum of the normalised rows --------------------------------------
   float acc[L::EPL];
 #pragma unroll
   for (int i = 0; i < L::EPL; ++i) acc[i] = 0.0f;
-  for (int r0 = lo + warp * L::RPW; r0 < hi; r0 += kRedWarps * L::RPW) {
-    const int r = r0 + sub;
-    const bool valid = r < hi;
-    float e[L::EPL];
-    if (valid) {
-      const uint4 u = ld_nc_v4(kh + (size_t)r * D + cl * L::EPL);
-      Vec16<T>::to_float(u, e);
-    } else {
+  for (int r0 = lo + warp * L::RPW * kRedUnroll; r0 < hi; r0 += kRowsPerIter) {
+    float e[kRedUnroll][L::EPL];
+    load_rows<T, D>(kh, r0, hi, sub, cl, e);
 #pragma unroll
-      for (int i = 0; i < L::EPL; ++i) e[i] = 0.0f;
+    for (int u = 0; u < kRedUnroll; ++u) {
+      float n2 = 0.0f;
+#pragma unroll
+      for (int i = 0; i < L::EPL; ++i) n2 = fmaf(e[u][i], e[u][i], n2);
+      n2 = row_sum<L::LPR>(n2);
+      const float inv = 1.0f / fmaxf(sqrtf(n2), 1e-12f);  // a zero key stays zero
+#pragma unroll
+      for (int i = 0; i < L::EPL; ++i) acc[i] = fmaf(e[u][i], inv, acc[i]);
     }
-    float n2 = 0.0f;
-#pragma unroll
-    for (int i = 0; i < L::EPL; ++i) n2 = fmaf(e[i], e[i], n2);
-    n2 = row_sum<L::LPR>(n2);
-    const float inv = 1.0f / fmaxf(sqrtf(n2), 1e-12f);  // a zero key stays zero
-#pragma unroll
-    for (int i = 0; i < L::EPL; ++i) acc[i] = fmaf(e[i], inv, acc[i]);
   }
-  // Reduce the rows of the warp: lanes with equal cl hold the same columns.
 #pragma unroll
   for (int o = L::LPR; o < 32; o <<= 1)
 #pragma unroll
     for (int i = 0; i < L::EPL; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-  __shared__ float s_acc[kRedWarps][D];
   if (sub == 0) {
 #pragma unroll
     for (int i = 0; i < L::EPL; ++i) s_acc[warp][cl * L::EPL + i] = acc[i];
@@ -98,128 +119,110 @@ __global__ void __launch_bounds__(kRedThreads)
     float t = 0.0f;
 #pragma unroll
     for (int w = 0; w < kRedWarps; ++w) t += s_acc[w][c];
-    partial_s[((size_t)h * bph + b) * D + c] = t;
+    s_part[c] = t;
   }
-}
-
-// Pass B: s = fixed-order sum of the partials, then e_j = exp(r_j) for this
-// block's rows; partial_e[h][b] = sum of this block's e_j.
-template <typename T, int D>
-__global__ void __launch_bounds__(kRedThreads)
-    red_dot_kernel(const T* __restrict__ k, int Lk, int bph, const float* __restrict__ partial_s,
-                   float* __restrict__ e_out, double* __restrict__ partial_e) {
-  using L = RowLayout<T, D>;
-  const int h = blockIdx.y, b = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane / L::LPR, cl = lane % L::LPR;
-  __shared__ float s_vec[D];
+  cluster.sync();
   for (int c = threadIdx.x; c < D; c += kRedThreads) {
     double t = 0.0;
-    for (int i = 0; i < bph; ++i) t += (double)partial_s[((size_t)h * bph + i) * D + c];
+    for (int q = 0; q < nrank; ++q) t += (double)*cluster.map_shared_rank(&s_part[c], q);
     s_vec[c] = (float)t;
   }
   __syncthreads();
+
+  // ---- 2. logits r_j and e_j = exp(r_j) -------------------------------------
   float sv[L::EPL];
 #pragma unroll
   for (int i = 0; i < L::EPL; ++i) sv[i] = s_vec[cl * L::EPL + i];
-
-  int lo, hi;
-  block_rows(Lk, bph, b, lo, hi);
-  const T* kh = k + (size_t)h * Lk * D;
   const float inv_lk = 1.0f / (float)Lk;
+  float* rh = red + (size_t)h * Lk;
   double esum = 0.0;
-  for (int r0 = lo + warp * L::RPW; r0 < hi; r0 += kRedWarps * L::RPW) {
-    const int r = r0 + sub;
-    const bool valid = r < hi;
-    float e[L::EPL];
-    if (valid) {
-      const uint4 u = ld_nc_v4(kh + (size_t)r * D + cl * L::EPL);
-      Vec16<T>::to_float(u, e);
-    } else {
+  for (int r0 = lo + warp * L::RPW * kRedUnroll; r0 < hi; r0 += kRowsPerIter) {
+    float e[kRedUnroll][L::EPL];
+    load_rows<T, D>(kh, r0, hi, sub, cl, e);
 #pragma unroll
-      for (int i = 0; i < L::EPL; ++i) e[i] = 0.0f;
-    }
-    float n2 = 0.0f, dot = 0.0f;
+    for (int u = 0; u < kRedUnroll; ++u) {
+      float n2 = 0.0f, dot = 0.0f;
 #pragma unroll
-    for (int i = 0; i < L::EPL; ++i) {
-      n2 = fmaf(e[i], e[i], n2);
-      dot = fmaf(e[i], sv[i], dot);
-    }
-    n2 = row_sum<L::LPR>(n2);
-    dot = row_sum<L::LPR>(dot);
-    const float inv = 1.0f / fmaxf(sqrtf(n2), 1e-12f);
-    // r_j = (khat_j . s - ||khat_j||^2) / L_k
-    const float rj = (dot * inv - n2 * inv * inv) * inv_lk;
-    const float ej = expf(rj);
-    if (valid && cl == 0) {
-      e_out[(size_t)h * Lk + r] = ej;
-      esum += (double)ej;
+      for (int i = 0; i < L::EPL; ++i) {
+        n2 = fmaf(e[u][i], e[u][i], n2);
+        dot = fmaf(e[u][i], sv[i], dot);
+      }
+      n2 = row_sum<L::LPR>(n2);
+      dot = row_sum<L::LPR>(dot);
+      const float inv = 1.0f / fmaxf(sqrtf(n2), 1e-12f);
+      // r_j = (khat_j . s - ||khat_j||^2) / L_k
+      const float rj = (dot * inv - n2 * inv * inv) * inv_lk;
+      const float ej = expf(rj);
+      const int r = r0 + u * L::RPW + sub;
+      if (r < hi && cl == 0) {
+        rh[r] = ej;
+        esum += (double)ej;
+      }
     }
   }
   esum = warp_sum(esum);
-  __shared__ double s_e[kRedWarps];
-  if (lane == 0) s_e[warp] = esum;
+  if (lane == 0) s_esum[warp] = esum;
   __syncthreads();
   if (threadIdx.x == 0) {
     double t = 0.0;
 #pragma unroll
-    for (int w = 0; w < kRedWarps; ++w) t += s_e[w];
-    partial_e[(size_t)h * bph + b] = t;
+    for (int w = 0; w < kRedWarps; ++w) t += s_esum[w];
+    s_epart = t;
   }
-}
-
-// Pass C: red = e / sum_j e_j.
-__global__ void __launch_bounds__(kRedThreads)
-    red_norm_kernel(float* __restrict__ red, int Lk, int bph, const double* __restrict__ partial_e) {
-  const int h = blockIdx.y;
-  __shared__ float s_inv;
+  cluster.sync();
   if (threadIdx.x == 0) {
-    double t = 0.0;
-    for (int i = 0; i < bph; ++i) t += partial_e[(size_t)h * bph + i];
-    s_inv = (float)(1.0 / t);
+    double z = 0.0;
+    for (int q = 0; q < nrank; ++q) z += *cluster.map_shared_rank(&s_epart, q);
+    s_inv = (float)(1.0 / z);
   }
-  __syncthreads();
+  cluster.sync();  // no CTA leaves while another may still read its shared memory
+
+  // ---- 3. normalise this CTA's rows ----------------------------------------------
   const float inv = s_inv;
-  float* rh = red + (size_t)h * Lk;
-  for (int j = blockIdx.x * kRedThreads + threadIdx.x; j < Lk; j += gridDim.x * kRedThreads)
-    rh[j] = rh[j] * inv;
+  for (int r = lo + threadIdx.x; r < hi; r += kRedThreads) rh[r] = rh[r] * inv;
 }
 
 template <typename T, int D>
-cudaError_t run(const T* k, int H, int Lk, float* red, char* ws, cudaStream_t s) {
-  using L = RowLayout<T, D>;
-  int bph = (int)ceil_div((int64_t)sm_count() * 4, H);
-  const int min_rows = kRedWarps * L::RPW * 4;  // at least four warp steps per block
-  bph = min(bph, (int)ceil_div(Lk, min_rows));
-  bph = max(1, min(bph, kRedMaxBlocksPerHead));
-  float* partial_s = reinterpret_cast<float*>(ws);
-  double* partial_e = reinterpret_cast<double*>(
-      ws + align_up((size_t)H * kRedMaxBlocksPerHead * D * sizeof(float), 256));
-  dim3 grid(bph, H);
-  red_sum_kernel<T, D><<<grid, kRedThreads, 0, s>>>(k, Lk, bph, partial_s);
-  red_dot_kernel<T, D><<<grid, kRedThreads, 0, s>>>(k, Lk, bph, partial_s, red, partial_e);
-  const int64_t nbc = ceil_div(Lk, kRedThreads);
-  dim3 gridc((unsigned)(nbc < 64 ? nbc : 64), H);
-  red_norm_kernel<<<gridc, kRedThreads, 0, s>>>(red, Lk, bph, partial_e);
-  return cudaGetLastError();
+cudaError_t run(const T* k, int H, int Lk, float* red, cudaStream_t s) {
+  // 16 CTAs per head when the slices stay long enough, else the portable 8.
+  const int csize = (Lk >= 16 * 64) ? 16 : 8;
+  auto kern = red_cluster_kernel<T, D>;
+  if (csize > 8) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)csize, (unsigned)H, 1);
+  cfg.blockDim = dim3(kRedThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, k, Lk, red);
 }
 }  // namespace
 
 size_t redundancy_ws_bytes(int H, int d) {
-  return align_up((size_t)H * kRedMaxBlocksPerHead * d * sizeof(float), 256) +
-         (size_t)H * kRedMaxBlocksPerHead * sizeof(double);
+  (void)H;
+  (void)d;
+  return 256;  // the fused kernel keeps its partial sums in (distributed) shared memory
 }
 
 cudaError_t launch_redundancy(const void* k, bool bf16, int H, int Lk, int d, float* red,
                               void* ws, cudaStream_t s) {
-  char* w = static_cast<char*>(ws);
+  (void)ws;
   if (bf16) {
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
-    return d == 128 ? run<__nv_bfloat16, 128>(kb, H, Lk, red, w, s)
-                    : run<__nv_bfloat16, 64>(kb, H, Lk, red, w, s);
+    return d == 128 ? run<__nv_bfloat16, 128>(kb, H, Lk, red, s)
+                    : run<__nv_bfloat16, 64>(kb, H, Lk, red, s);
   }
   const float* kf = static_cast<const float*>(k);
-  return d == 128 ? run<float, 128>(kf, H, Lk, red, w, s) : run<float, 64>(kf, H, Lk, red, w, s);
+  return d == 128 ? run<float, 128>(kf, H, Lk, red, s) : run<float, 64>(kf, H, Lk, red, s);
 }
 
 }  // namespace fc
