@@ -43,8 +43,9 @@ def flush_l2(buf, sink):
     starts with a clean L2 (no write-back traffic of ours lands on it)."""
     buf.zero_()
     torch.sum(buf.view(torch.float32), dim=0, out=sink)
-# Kernel launches per call, as implemented in cache_gating_kv_b200/csrc.
-LAUNCHES = {"gate": 1, "importance": 2, "redundancy": 1, "score_topb": 2, "compact": 1}
+# Kernel launches per call, as implemented in cache_gating_kv_b200/csrc (importance:
+# row pass, key-split merge, column pass -- the split is taken on 148-SM B200s).
+LAUNCHES = {"gate": 1, "importance": 3, "redundancy": 1, "score_topb": 2, "compact": 1}
 
 
 def _args():

@@ -51,17 +51,20 @@ namespace {
 constexpr int kBM = 128;      // rows of the resident A tile (TMEM lanes)
 constexpr int kBN = 128;      // rows of each streamed B tile (MMA N, TMEM columns)
 constexpr int kStages = 4;    // shared-memory ring depth
-constexpr int kAcc = 4;       // TMEM accumulators of kBN columns
-constexpr int kThreads = 384;
+constexpr int kAcc = 4;       // TMEM accumulators of kBN columns (all 512 columns)
+constexpr int kEpi = 3;       // epilogue warpgroups; tile t goes to group t % kEpi
+constexpr int kThreads = 128 + 128 * kEpi;
+constexpr int kCh = 32;       // TMEM columns per tcgen05.ld chunk
 constexpr int kHalf = kBM * 64 * 2;  // one 128 x 64 bf16 swizzled block (16 KB)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr size_t kErrOffset = 0;      // error word in the workspace
-constexpr size_t kLseOffset = 256;    // nl [H][Lq_pad] follows
+constexpr size_t kLseOffset = 256;    // nl [H][Lq_pad] follows, then the split partials
+constexpr int kMaxSplit = 4;          // pass 1 may split the key range in up to 4 parts
 constexpr float kRescaleAt = 4294967296.0f;  // 2^32
 
-// Which pairs of a 64-column half go to the FMA pipes: 3 of every 8 values.
+// Which pairs of a 32-column chunk go to the FMA pipes: 6 of 16 (3/8).
 __device__ __forceinline__ constexpr bool emulated_pair(int p) {
-  return (p & 3) == 1 || (p & 7) == 6;
+  return (p & 7) == 1 || (p & 7) == 4 || (p & 7) == 6;
 }
 
 template <int D>
@@ -71,7 +74,7 @@ constexpr int tile_bytes() {
 template <int D>
 constexpr size_t smem_bytes() {
   return 1024 + (size_t)(1 + kStages) * tile_bytes<D>() + 256 + kStages * kBN * sizeof(float) +
-         2 * kBM * sizeof(float);
+         2 * kEpi * kBM * sizeof(float);
 }
 
 struct Bars {
@@ -84,54 +87,90 @@ struct Bars {
 };
 
 __device__ __forceinline__ void epilogue_sync() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");  // the 8 epilogue warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(128 * kEpi) : "memory");  // the epilogue warps only
 }
 
 __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) {
   return make_float2(__uint_as_float(a), __uint_as_float(b));
 }
 
-// Sum of 2^(c*s - ref) over 64 values; mixes MUFU and FMA-pipe exponentials.
-template <bool kClampHigh>
-__device__ __forceinline__ float half_sum_shifted(const uint32_t (&r)[64], float c, float ref) {
+__device__ __forceinline__ float2 exp2_pair(int p, float2 x, bool clamp_high) {
+  if (emulated_pair(p)) return clamp_high ? tc::ex2_poly2<true>(x) : tc::ex2_poly2<false>(x);
+  return make_float2(tc::ex2(x.x), tc::ex2(x.y));
+}
+
+// Sum of 2^(c*s - ref) over one chunk; mixes MUFU and FMA-pipe exponentials.
+__device__ __forceinline__ float chunk_sum_shifted(const uint32_t (&r)[kCh], float c, float ref) {
   const float2 cc = make_float2(c, c), sh = make_float2(-ref, -ref);
-  float2 acc0 = make_float2(0.f, 0.f), acc1 = make_float2(0.f, 0.f);
+  float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
-  for (int p = 0; p < 32; ++p) {
-    const float2 x = tc::ffma2(f2(r[2 * p], r[2 * p + 1]), cc, sh);
-    float2 e;
-    if (emulated_pair(p)) {
-      e = tc::ex2_poly2<kClampHigh>(x);
-    } else {
-      e.x = tc::ex2(x.x);
-      e.y = tc::ex2(x.y);
-    }
+  for (int p = 0; p < kCh / 2; ++p) {
+    const float2 e = exp2_pair(p, tc::ffma2(f2(r[2 * p], r[2 * p + 1]), cc, sh), true);
     if (p & 1)
-      acc1 = tc::fadd2(acc1, e);
+      a1 = tc::fadd2(a1, e);
     else
-      acc0 = tc::fadd2(acc0, e);
+      a0 = tc::fadd2(a0, e);
   }
-  const float2 a = tc::fadd2(acc0, acc1);
+  const float2 a = tc::fadd2(a0, a1);
   return a.x + a.y;
 }
 
-__device__ __forceinline__ float half_max(const uint32_t (&r)[64]) {
+__device__ __forceinline__ float chunk_max(const uint32_t (&r)[kCh]) {
   float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < 64; j += 4) {
+  for (int j = 0; j < kCh; j += 4) {
     m0 = tc::fmax3(m0, __uint_as_float(r[j]), __uint_as_float(r[j + 1]));
     m1 = tc::fmax3(m1, __uint_as_float(r[j + 2]), __uint_as_float(r[j + 3]));
   }
   return fmaxf(m0, m1);
 }
 
-// kPass 1: A = Q tile, B = K tiles, epilogue = row log-sum-exp.
+// Pass 1 on one chunk: mask keys past L_k, then fold the chunk into the row's
+// (reference, sum) pair.  The reference lags the running max: it only moves
+// when the chunk's sum passes 2^32, and then exactly (rescale, recompute).
+__device__ __forceinline__ void row_chunk(uint32_t (&r)[kCh], int valid, float c2, float& ref,
+                                          float& l) {
+  if (valid < kCh) {
+#pragma unroll
+    for (int j = 0; j < kCh; ++j)
+      if (j >= valid) r[j] = 0xff800000u;  // -inf
+  }
+  if (ref == -INFINITY) ref = chunk_max(r) * c2;  // first values this group sees
+  if (ref == -INFINITY) return;                   // every key here was padding
+  float cs = chunk_sum_shifted(r, c2, ref);
+  if (!(cs <= kRescaleAt)) {
+    const float rnew = fmaxf(ref, chunk_max(r) * c2);
+    l *= tc::ex2(ref - rnew);
+    ref = rnew;
+    cs = chunk_sum_shifted(r, c2, ref);
+  }
+  l += cs;
+}
+
+// Pass 2 on one chunk: acc += 2^(c*s + nl_q) over the chunk's 32 queries.
+__device__ __forceinline__ void col_chunk(const uint32_t (&r)[kCh], const float* __restrict__ nlc,
+                                          float c2, float2& acc) {
+  const float2 cc = make_float2(c2, c2);
+  const float2* L2 = reinterpret_cast<const float2*>(nlc);
+  float2 a1 = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int p = 0; p < kCh / 2; ++p) {
+    const float2 e = exp2_pair(p, tc::ffma2(f2(r[2 * p], r[2 * p + 1]), cc, L2[p]), false);
+    if (p & 1)
+      a1 = tc::fadd2(a1, e);
+    else
+      acc = tc::fadd2(acc, e);
+  }
+  acc = tc::fadd2(acc, a1);
+}
+
+// kPass 1: A = Q tile, B = K tiles of one key split, epilogue = row log-sum-exp.
 // kPass 2: A = K tile, B = Q tiles, epilogue = column sums of 2^(c s + nl).
 template <int D, int kPass>
 __global__ void __launch_bounds__(kThreads, 1)
     imp_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                  int Lq, int Lk, int lq_pad, float c2, float* __restrict__ nl,
-                  float* __restrict__ imp, int* __restrict__ err) {
+                  int Lq, int Lk, int lq_pad, int nsplit, float c2, float* __restrict__ nl,
+                  float2* __restrict__ part, float* __restrict__ imp, int* __restrict__ err) {
   constexpr int KB = D / 64;
   constexpr int TB = tile_bytes<D>();
   constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kBM, kBN);
@@ -142,12 +181,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sB = base + TB;
   Bars* bars = reinterpret_cast<Bars*>(sB + kStages * TB);
   float* sL = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // [kStages][kBN]
-  float* sM = sL + kStages * kBN;  // [2][kBM] merge buffer of the two warpgroups
+  float* sM = sL + kStages * kBN;  // [2*kEpi][kBM] merge buffer of the epilogue groups
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
-  const int a0 = blockIdx.x * kBM;  // first row of the A tile
-  const int nB = kPass == 1 ? (Lk + kBN - 1) / kBN : lq_pad / kBN;
+  const int unit = kPass == 1 ? blockIdx.x / nsplit : blockIdx.x;
+  const int split = kPass == 1 ? blockIdx.x % nsplit : 0;
+  const int a0 = unit * kBM;  // first row of the A tile
+  int t_begin = 0, nB;
+  if (kPass == 1) {
+    const int nkt = (Lk + kBN - 1) / kBN;
+    const int per = (nkt + nsplit - 1) / nsplit;
+    t_begin = split * per;
+    nB = min(nkt, t_begin + per) - t_begin;
+  } else {
+    nB = lq_pad / kBN;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -182,10 +231,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc::mbar_expect_tx(&bars->full[s], TB + (kPass == 2 ? kBN * 4 : 0));
+        const int row_b = (t_begin + t) * kBN;
         for (int kb = 0; kb < KB; ++kb)
-          tc::tma_load_3d(sB + s * TB + kb * kHalf, &mapB, &bars->full[s], kb * 64, t * kBN, h);
+          tc::tma_load_3d(sB + s * TB + kb * kHalf, &mapB, &bars->full[s], kb * 64, row_b, h);
         if (kPass == 2)
-          tc::bulk_load(sL + s * kBN, nl + (size_t)h * lq_pad + t * kBN, kBN * 4, &bars->full[s]);
+          tc::bulk_load(sL + s * kBN, nl + (size_t)h * lq_pad + row_b, kBN * 4, &bars->full[s]);
       }
     }
   } else if (warp == 1) {
@@ -211,14 +261,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mma_commit(&bars->acc_full[b]);  // accumulator b ready
       }
     }
-  } else if (warp >= 4) {  // ---- two epilogue warpgroups, tiles alternate between them
-    const int g = (warp - 4) >> 2;   // warpgroup 0 takes even tiles, 1 odd tiles
-    const int sub = warp & 3;        // TMEM lane quarter
+  } else if (warp >= 4) {  // ---- kEpi epilogue warpgroups; tile t goes to group t % kEpi
+    const int g = (warp - 4) >> 2;
+    const int sub = warp & 3;          // TMEM lane quarter
     const int rloc = sub * 32 + lane;  // this thread's row of the A tile
     const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
-    float ref = -INFINITY, l = 0.0f;  // pass 1: running reference and sum (log2 units)
-    float2 acc = make_float2(0.f, 0.f);  // pass 2: column sum (two chains)
-    for (int t = g; t < nB; t += 2) {
+    float ref = -INFINITY, l = 0.0f;     // pass 1: reference and sum (log2 units)
+    float2 acc = make_float2(0.f, 0.f);  // pass 2: column sum
+    for (int t = g; t < nB; t += kEpi) {
       const int b = t % kAcc, v = t / kAcc, s = t % kStages, u = t / kStages;
       if (!tc::mbar_wait(&bars->acc_full[b], v & 1) ||
           (kPass == 2 && !tc::mbar_wait(&bars->full[s], u & 1))) {
@@ -226,86 +276,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       tc::fence_after_sync();
+      const uint32_t col0 = lane_addr + b * kBN;
+      const int valid = Lk - (t_begin + t) * kBN;  // pass 1: keys left in this tile
+      const float* nlt = sL + s * kBN;             // pass 2: this tile's nl values
+      // Four chunks of 32 columns; chunk c+1's TMEM load is in flight while
+      // chunk c is being computed.
+      uint32_t ra[kCh], rb[kCh];
+      tc::tmem_ld32(col0, ra);
+      tc::tmem_ld_wait(ra);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t r[64];
-        tc::tmem_ld32(lane_addr + b * kBN + hf * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
-        tc::tmem_ld32(lane_addr + b * kBN + hf * 64 + 32,
-                      *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-        tc::tmem_ld_wait();
-        if (hf == 1) {
+      for (int c = 0; c < kBN / kCh; c += 2) {
+        tc::tmem_ld32(col0 + (c + 1) * kCh, rb);
+        if (kPass == 1)
+          row_chunk(ra, valid - c * kCh, c2, ref, l);
+        else
+          col_chunk(ra, nlt + c * kCh, c2, acc);
+        tc::tmem_ld_wait(rb);
+        if (c + 2 < kBN / kCh) {
+          tc::tmem_ld32(col0 + (c + 2) * kCh, ra);
+        } else {
           tc::fence_before_sync();
           __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&bars->acc_empty[b]);  // values are in registers
+          if (lane == 0) tc::mbar_arrive(&bars->acc_empty[b]);  // every column is in registers
         }
-        if (kPass == 1) {
-          const int valid = Lk - t * kBN - hf * 64;  // >= 64 except near the end
-          if (valid < 64) {
-#pragma unroll
-            for (int j = 0; j < 64; ++j)
-              if (j >= valid) r[j] = 0xff800000u;  // -inf: a key past L_k
-          }
-          if (ref == -INFINITY) ref = half_max(r) * c2;  // first values this group sees
-          if (ref != -INFINITY) {
-            float hs = half_sum_shifted<true>(r, c2, ref);
-            if (!(hs <= kRescaleAt)) {  // much larger logits arrived: move the reference
-              const float rnew = fmaxf(ref, half_max(r) * c2);
-              l *= tc::ex2(ref - rnew);
-              ref = rnew;
-              hs = half_sum_shifted<true>(r, c2, ref);
-            }
-            l += hs;
-          }
-        } else {
-          const float2* L2 = reinterpret_cast<const float2*>(sL + s * kBN + hf * 64);
-          const float2 cc = make_float2(c2, c2);
-          float2 acc1 = make_float2(0.f, 0.f);
-#pragma unroll
-          for (int p = 0; p < 32; ++p) {
-            const float2 x = tc::ffma2(f2(r[2 * p], r[2 * p + 1]), cc, L2[p]);
-            float2 e;
-            if (emulated_pair(p)) {
-              e = tc::ex2_poly2<false>(x);
-            } else {
-              e.x = tc::ex2(x.x);
-              e.y = tc::ex2(x.y);
-            }
-            if (p & 1)
-              acc1 = tc::fadd2(acc1, e);
-            else
-              acc = tc::fadd2(acc, e);
-          }
-          acc = tc::fadd2(acc, acc1);
-        }
+        if (kPass == 1)
+          row_chunk(rb, valid - (c + 1) * kCh, c2, ref, l);
+        else
+          col_chunk(rb, nlt + (c + 1) * kCh, c2, acc);
+        if (c + 2 < kBN / kCh) tc::tmem_ld_wait(ra);
       }
       if (kPass == 2) {
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bars->empty[s]);  // done with this stage's nl values
       }
     }
-    // Merge the two warpgroups' partial results for each row (both groups
-    // always reach this barrier, also after a timeout).
-    if (kPass == 1) {
-      if (g == 1) {
-        sM[rloc] = ref;      // group 1's reference
-        sM[kBM + rloc] = l;  // group 1's sum
-      }
-      epilogue_sync();
-      if (g == 0 && ok) {
-        const float r1 = sM[rloc], l1 = sM[kBM + rloc];
-        const float M = fmaxf(ref, r1);
-        float L = 0.0f;
-        if (ref != -INFINITY) L += l * tc::ex2(ref - M);
-        if (r1 != -INFINITY) L += l1 * tc::ex2(r1 - M);
-        const int row = a0 + rloc;
-        nl[(size_t)h * lq_pad + row] = row < Lq ? -(M + __log2f(L)) : -INFINITY;
-      }
-    } else {
-      if (g == 1) sM[rloc] = acc.x + acc.y;
-      epilogue_sync();
-      if (g == 0 && ok) {
-        const int row = a0 + rloc;
-        if (row < Lk) imp[(size_t)h * Lk + row] = ((acc.x + acc.y) + sM[rloc]) / (float)Lq;
+    // Merge the groups' partial results for each row (every group reaches
+    // this barrier, also after a timeout).
+    if (g > 0) {
+      sM[(2 * g) * kBM + rloc] = kPass == 1 ? ref : acc.x + acc.y;
+      sM[(2 * g + 1) * kBM + rloc] = l;
+    }
+    epilogue_sync();
+    if (g == 0 && ok) {
+      const int row = a0 + rloc;
+      if (kPass == 1) {
+        float M = ref;
+#pragma unroll
+        for (int q = 1; q < kEpi; ++q) M = fmaxf(M, sM[(2 * q) * kBM + rloc]);
+        float L = (ref == -INFINITY) ? 0.0f : l * tc::ex2(ref - M);
+#pragma unroll
+        for (int q = 1; q < kEpi; ++q) {
+          const float rq = sM[(2 * q) * kBM + rloc];
+          if (rq != -INFINITY) L += sM[(2 * q + 1) * kBM + rloc] * tc::ex2(rq - M);
+        }
+        if (nsplit == 1)
+          nl[(size_t)h * lq_pad + row] = row < Lq ? -(M + __log2f(L)) : -INFINITY;
+        else
+          part[((size_t)split * gridDim.y + h) * lq_pad + row] = make_float2(M, L);
+      } else {
+        float sum = acc.x + acc.y;
+#pragma unroll
+        for (int q = 1; q < kEpi; ++q) sum += sM[(2 * q) * kBM + rloc];
+        if (row < Lk) imp[(size_t)h * Lk + row] = sum / (float)Lq;
       }
     }
   }
@@ -314,6 +346,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::fence_after_sync();
   if (warp == 2) tc::tmem_dealloc(tmem, kAcc * kBN);
+}
+
+// Combine the key-split partial (reference, sum) pairs of every query row.
+__global__ void nl_merge_kernel(const float2* __restrict__ part, int nsplit, int H, int Lq,
+                                int lq_pad, float* __restrict__ nl) {
+  const int64_t n = (int64_t)H * lq_pad;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int row = (int)(i % lq_pad);
+    float M = -INFINITY;
+    for (int q = 0; q < nsplit; ++q) M = fmaxf(M, part[q * n + i].x);
+    float L = 0.0f;
+    for (int q = 0; q < nsplit; ++q) {
+      const float2 p = part[q * n + i];
+      if (p.x != -INFINITY) L += p.y * tc::ex2(p.x - M);
+    }
+    nl[i] = row < Lq ? -(M + __log2f(L)) : -INFINITY;
+  }
+}
+
+// Key splits for pass 1: the fewest (<= kMaxSplit) whose grid wastes at most
+// 10 % of the last wave, keeping >= 8 key tiles per split.
+int choose_split(int units, int nkt) {
+  const int sms = sm_count();
+  int best = 1;
+  double best_eff = 0.0;
+  for (int s = 1; s <= kMaxSplit; ++s) {
+    if (s > 1 && nkt / s < 8) break;
+    const double n = (double)units * s;
+    const double eff = n / (ceil_div((int64_t)n, sms) * (double)sms);
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = s;
+    }
+    if (eff >= 0.90) break;
+  }
+  return best;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -354,8 +423,10 @@ cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, float scale
   CUtensorMap mq, mk;
   if (!make_map(&mq, q, H, Lq, D) || !make_map(&mk, k, H, Lk, D)) return cudaErrorInvalidValue;
   int* err = reinterpret_cast<int*>(static_cast<char*>(ws) + kErrOffset);
-  float* nl = reinterpret_cast<float*>(static_cast<char*>(ws) + kLseOffset);
   const int lq_pad = (int)ceil_div(Lq, kBM) * kBM;
+  float* nl = reinterpret_cast<float*>(static_cast<char*>(ws) + kLseOffset);
+  float2* part = reinterpret_cast<float2*>(
+      static_cast<char*>(ws) + kLseOffset + align_up((size_t)H * lq_pad * sizeof(float), 256));
   const float c2 = scale * kLog2e;
   const size_t smem = smem_bytes<D>();
   cudaError_t e;
@@ -365,10 +436,19 @@ cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, float scale
   e = cudaFuncSetAttribute(imp_tc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  imp_tc_kernel<D, 1><<<dim3(lq_pad / kBM, H), kThreads, smem, s>>>(mq, mk, Lq, Lk, lq_pad, c2,
-                                                                     nl, imp, err);
+  const int nq = lq_pad / kBM;
+  const int nkt = (int)ceil_div(Lk, kBN);
+  const int nsplit = choose_split(nq * H, nkt);
+  imp_tc_kernel<D, 1><<<dim3(nq * nsplit, H), kThreads, smem, s>>>(
+      mq, mk, Lq, Lk, lq_pad, nsplit, c2, nl, part, imp, err);
+  if (nsplit > 1) {
+    const int64_t n = (int64_t)H * lq_pad;
+    const int64_t blocks = ceil_div(n, 256);
+    nl_merge_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(part, nsplit, H, Lq,
+                                                                            lq_pad, nl);
+  }
   imp_tc_kernel<D, 2><<<dim3((unsigned)ceil_div(Lk, kBM), H), kThreads, smem, s>>>(
-      mk, mq, Lq, Lk, lq_pad, c2, nl, imp, err);
+      mk, mq, Lq, Lk, lq_pad, 1, c2, nl, part, imp, err);
   return cudaGetLastError();
 }
 
@@ -387,7 +467,8 @@ __global__ void exp2_selftest_kernel(const float* x, float* y_mufu, float* y_pol
 }  // namespace
 
 size_t importance_ws_bytes(int H, int Lq) {
-  return kLseOffset + align_up((size_t)H * ceil_div(Lq, kBM) * kBM * sizeof(float), 256);
+  const size_t rows = (size_t)H * ceil_div(Lq, kBM) * kBM;
+  return kLseOffset + align_up(rows * sizeof(float), 256) + kMaxSplit * rows * sizeof(float2);
 }
 
 bool importance_tc_supported(int d) { return d == 64 || d == 128; }
