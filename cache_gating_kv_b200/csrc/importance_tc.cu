@@ -6,39 +6,48 @@
 //
 // The L_q x L_k probability matrix is never stored.  Two passes recompute the
 // logits with tcgen05.mma:
-//   pass 1 (rows)     CTA = 128 queries of one head; streams every 128-key
+//   pass 1 (rows)     CTA = 128 queries of one head; streams every 256-key
 //                     tile; D = Q K^T in TMEM; the epilogue thread that owns a
 //                     query row keeps a (reference, sum) pair in log2 units
 //                     and the CTA writes nl_q = -log2 sum_j 2^(c s_qj),
 //                     c = scale*log2(e) (padded query rows: -inf).
-//   pass 2 (columns)  CTA = 128 keys of one head; streams every 128-query tile;
+//   pass 2 (columns)  CTA = 128 keys of one head; streams every 256-query tile;
 //                     D = K Q^T in TMEM (keys on the TMEM lanes), so each
 //                     epilogue thread owns one key and sums 2^(c s + nl_q)
 //                     over all queries in registers: no atomics, no partial
 //                     buffers, deterministic.
 //
 // Work per score is one tensor-core MAC row (256 flops at d=128) and one
-// exponential.  The SM's special-function unit retires 16 exponentials per
+// exponential.  The SM's special-function unit retires ~16 exponentials per
 // clock against ~32 scores per clock of dense bf16 MMA, so the epilogue, not
 // the MMA, sets the pace.  The design therefore
-//   - runs two epilogue warpgroups in ping-pong over four 128-column TMEM
-//     accumulators (the tensor core fills tile t+2 while tiles t and t+1 are
-//     being drained);
+//   - issues M=128, N=256, K=16 MMAs: at N=128 the single-CTA MMA is bound by
+//     reading its operands from shared memory (measured ~1.0 PFLOP/s with the
+//     epilogue and TMA removed); N=256 reuses each A fragment for twice the
+//     columns;
+//   - keeps two 256-column TMEM accumulators in flight and lets every
+//     epilogue warpgroup drain its own 64-column slice of every tile: an
+//     accumulator is handed back to the MMA as soon as each warp has loaded
+//     its slice;
 //   - uses packed f32x2 FMA/ADD for the scale-and-shift and the running sums;
-//   - evaluates 3 of every 8 exponentials on the FMA pipes (ex2_poly2, a
-//     polynomial of our own) and the rest on the special-function unit;
+//   - evaluates 1 of every 4 exponentials on the FMA pipes (ex2_poly2, a
+//     polynomial of our own) and the rest on the special-function unit (a
+//     sweep of the mix on B200 put the optimum there);
 //   - in pass 1 shifts by a lagged reference instead of the exact running max:
-//     the reference only moves (with an exact rescale) when a half tile's sum
-//     exceeds 2^32, so the per-element max disappears from the common path.
+//     the reference only moves (with an exact rescale) when a chunk's sum
+//     exceeds 2^32, so the per-element max disappears from the common path;
+//   - in pass 1 splits the key range in 2-4 parts when that fills the last
+//     wave of CTAs better; a small kernel merges the partial (reference, sum)
+//     pairs.
 //
-// Roles (384 threads): warp 0 lane 0 issues TMA loads (3D tensor maps over
+// Roles (640 threads): warp 0 lane 0 issues TMA loads (3D tensor maps over
 // [H][L][d], 128-byte swizzle, zero fill past L, no multicast), warp 1 lane 0
-// issues the MMAs (M=128, N=128, K=16 steps), warp 2 owns the TMEM allocation
-// (all 512 columns), warps 4-7 and 8-11 are the two epilogue warpgroups (warp
-// w reads TMEM lanes 32(w%4)..+31).  A shared-memory ring of operand tiles
-// decouples TMA from the MMAs.  Every mbarrier wait is bounded; on timeout the
-// kernel records an error word in the workspace and winds down (no trap, no
-// endless spin).
+// issues the MMAs (M=128, N=256, K=16 steps), warp 2 owns the TMEM allocation
+// (all 512 columns), warps 4-19 are four epilogue warpgroups (warp w reads
+// TMEM lanes 32(w%4)..+31).  A two-stage shared-memory ring of 64 KB operand
+// tiles decouples TMA from the MMAs.  Every mbarrier wait is bounded; on timeout the kernel
+// records an error word in the workspace and winds down (no trap, no endless
+// spin).
 #include <cuda.h>
 
 #include "fc_common.cuh"
@@ -48,33 +57,46 @@
 namespace fc {
 
 namespace {
-constexpr int kBM = 128;      // rows of the resident A tile (TMEM lanes)
-constexpr int kBN = 128;      // rows of each streamed B tile (MMA N, TMEM columns)
-constexpr int kStages = 4;    // shared-memory ring depth
-constexpr int kAcc = 4;       // TMEM accumulators of kBN columns (all 512 columns)
-constexpr int kEpi = 3;       // epilogue warpgroups; tile t goes to group t % kEpi
+constexpr int kBM = 128;      // rows of the resident A tile (MMA M, TMEM lanes)
+constexpr int kBN = 256;      // rows of each streamed B tile (MMA N, TMEM columns)
+constexpr int kStages = 2;    // shared-memory ring depth (64 KB B tiles)
+constexpr int kAcc = 2;       // TMEM accumulators of kBN columns (all 512 columns)
+#ifndef FC_IMP_EPI
+#define FC_IMP_EPI 4
+#endif
+#ifndef FC_IMP_EMU_MASK
+#define FC_IMP_EMU_MASK 0x2222  // pairs 1, 5, 9, 13 of 16: 1/4 of the exponentials
+#endif
+constexpr int kEpi = FC_IMP_EPI;  // epilogue warpgroups; each owns kBN/kEpi columns of every tile
 constexpr int kThreads = 128 + 128 * kEpi;
 constexpr int kCh = 32;       // TMEM columns per tcgen05.ld chunk
-constexpr int kHalf = kBM * 64 * 2;  // one 128 x 64 bf16 swizzled block (16 KB)
+constexpr int kSlice = kBN / kEpi;  // columns of a tile that one epilogue group drains
+static_assert(kSlice % kCh == 0, "each group drains whole chunks");
+constexpr int kHalfA = kBM * 64 * 2;  // one 128-row x 64-element bf16 swizzled block (16 KB)
+constexpr int kHalfB = kBN * 64 * 2;  // one 256-row x 64-element bf16 swizzled block (32 KB)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr size_t kErrOffset = 0;      // error word in the workspace
 constexpr size_t kLseOffset = 256;    // nl [H][Lq_pad] follows, then the split partials
 constexpr int kMaxSplit = 4;          // pass 1 may split the key range in up to 4 parts
 constexpr float kRescaleAt = 4294967296.0f;  // 2^32
 
-// Which pairs of a 32-column chunk go to the FMA pipes: 6 of 16 (3/8).
+// Which pairs of a 32-column chunk go to the FMA pipes (bit p of the mask).
 __device__ __forceinline__ constexpr bool emulated_pair(int p) {
-  return (p & 7) == 1 || (p & 7) == 4 || (p & 7) == 6;
+  return ((FC_IMP_EMU_MASK >> p) & 1) != 0;
 }
 
 template <int D>
-constexpr int tile_bytes() {
-  return (D / 64) * kHalf;
+constexpr int a_bytes() {
+  return (D / 64) * kHalfA;
+}
+template <int D>
+constexpr int b_bytes() {
+  return (D / 64) * kHalfB;
 }
 template <int D>
 constexpr size_t smem_bytes() {
-  return 1024 + (size_t)(1 + kStages) * tile_bytes<D>() + 256 + kStages * kBN * sizeof(float) +
-         2 * kEpi * kBM * sizeof(float);
+  return 1024 + (size_t)a_bytes<D>() + (size_t)kStages * b_bytes<D>() + 256 +
+         kStages * kBN * sizeof(float) + 2 * kEpi * kBM * sizeof(float);
 }
 
 struct Bars {
@@ -172,13 +194,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                   int Lq, int Lk, int lq_pad, int nsplit, float c2, float* __restrict__ nl,
                   float2* __restrict__ part, float* __restrict__ imp, int* __restrict__ err) {
   constexpr int KB = D / 64;
-  constexpr int TB = tile_bytes<D>();
+  constexpr int TA = a_bytes<D>();
+  constexpr int TB = b_bytes<D>();
   constexpr uint32_t kIdesc = tc::idesc_bf16_f32(kBM, kBN);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
   uint8_t* sA = base;
-  uint8_t* sB = base + TB;
+  uint8_t* sB = base + TA;
   Bars* bars = reinterpret_cast<Bars*>(sB + kStages * TB);
   float* sL = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // [kStages][kBN]
   float* sM = sL + kStages * kBN;  // [2*kEpi][kBM] merge buffer of the epilogue groups
@@ -202,13 +225,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       tc::mbar_init(&bars->full[s], 1);
       // pass 2: a stage also carries the query tile's nl values, so it is
-      // released by the MMA commit and by the 4 warps of the consuming group
-      tc::mbar_init(&bars->empty[s], kPass == 2 ? 5 : 1);
+      // released by the MMA commit and by every epilogue warp
+      tc::mbar_init(&bars->empty[s], kPass == 2 ? 1 + 4 * kEpi : 1);
     }
     tc::mbar_init(&bars->a_full, 1);
     for (int b = 0; b < kAcc; ++b) {
       tc::mbar_init(&bars->acc_full[b], 1);
-      tc::mbar_init(&bars->acc_empty[b], 4);
+      tc::mbar_init(&bars->acc_empty[b], 4 * kEpi);  // every epilogue warp reads its slice
     }
     tc::fence_barrier_init();
   }
@@ -221,9 +244,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {  // ---- TMA producer
-      tc::mbar_expect_tx(&bars->a_full, TB);
+      tc::mbar_expect_tx(&bars->a_full, TA);
       for (int kb = 0; kb < KB; ++kb)
-        tc::tma_load_3d(sA + kb * kHalf, &mapA, &bars->a_full, kb * 64, a0, h);
+        tc::tma_load_3d(sA + kb * kHalfA, &mapA, &bars->a_full, kb * 64, a0, h);
       for (int t = 0; t < nB; ++t) {
         const int s = t % kStages, u = t / kStages;
         if (!tc::mbar_wait(&bars->empty[s], (u & 1) ^ 1)) {
@@ -233,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::mbar_expect_tx(&bars->full[s], TB + (kPass == 2 ? kBN * 4 : 0));
         const int row_b = (t_begin + t) * kBN;
         for (int kb = 0; kb < KB; ++kb)
-          tc::tma_load_3d(sB + s * TB + kb * kHalf, &mapB, &bars->full[s], kb * 64, row_b, h);
+          tc::tma_load_3d(sB + s * TB + kb * kHalfB, &mapB, &bars->full[s], kb * 64, row_b, h);
         if (kPass == 2)
           tc::bulk_load(sL + s * kBN, nl + (size_t)h * lq_pad + row_b, kBN * 4, &bars->full[s]);
       }
@@ -253,22 +276,23 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t b_addr = tc::smem_u32(sB + s * TB);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kHalf + (kk & 3) * 32;  // 16 bf16 = 32 bytes per step
-          tc::mma_bf16(tmem + b * kBN, tc::desc_k_sw128(a_addr + off),
-                       tc::desc_k_sw128(b_addr + off), kIdesc, kk > 0 ? 1u : 0u);
+          const uint32_t ks = (kk & 3) * 32;  // 16 bf16 = 32 bytes per K step
+          tc::mma_bf16(tmem + b * kBN, tc::desc_k_sw128(a_addr + (kk >> 2) * kHalfA + ks),
+                       tc::desc_k_sw128(b_addr + (kk >> 2) * kHalfB + ks), kIdesc,
+                       kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(&bars->empty[s]);     // operand stage reusable once read
         tc::mma_commit(&bars->acc_full[b]);  // accumulator b ready
       }
     }
-  } else if (warp >= 4) {  // ---- kEpi epilogue warpgroups; tile t goes to group t % kEpi
+  } else if (warp >= 4) {  // ---- kEpi epilogue warpgroups, each on its column slice
     const int g = (warp - 4) >> 2;
     const int sub = warp & 3;          // TMEM lane quarter
     const int rloc = sub * 32 + lane;  // this thread's row of the A tile
-    const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
+    const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16) + g * kSlice;
     float ref = -INFINITY, l = 0.0f;     // pass 1: reference and sum (log2 units)
     float2 acc = make_float2(0.f, 0.f);  // pass 2: column sum
-    for (int t = g; t < nB; t += kEpi) {
+    for (int t = 0; t < nB; ++t) {
       const int b = t % kAcc, v = t / kAcc, s = t % kStages, u = t / kStages;
       if (!tc::mbar_wait(&bars->acc_full[b], v & 1) ||
           (kPass == 2 && !tc::mbar_wait(&bars->full[s], u & 1))) {
@@ -277,33 +301,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc::fence_after_sync();
       const uint32_t col0 = lane_addr + b * kBN;
-      const int valid = Lk - (t_begin + t) * kBN;  // pass 1: keys left in this tile
-      const float* nlt = sL + s * kBN;             // pass 2: this tile's nl values
-      // Four chunks of 32 columns; chunk c+1's TMEM load is in flight while
-      // chunk c is being computed.
-      uint32_t ra[kCh], rb[kCh];
-      tc::tmem_ld32(col0, ra);
-      tc::tmem_ld_wait(ra);
+      const int valid = Lk - (t_begin + t) * kBN - g * kSlice;  // pass 1: keys left
+      const float* nlt = sL + s * kBN + g * kSlice;             // pass 2: nl of the slice
 #pragma unroll
-      for (int c = 0; c < kBN / kCh; c += 2) {
-        tc::tmem_ld32(col0 + (c + 1) * kCh, rb);
+      for (int c = 0; c < kSlice / kCh; ++c) {
+        uint32_t ra[kCh];
+        tc::tmem_ld32(col0 + c * kCh, ra);
+        tc::tmem_ld_wait(ra);
+        if (c + 1 == kSlice / kCh) {  // the slice is in registers: free the accumulator
+          tc::fence_before_sync();
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&bars->acc_empty[b]);
+        }
         if (kPass == 1)
           row_chunk(ra, valid - c * kCh, c2, ref, l);
         else
           col_chunk(ra, nlt + c * kCh, c2, acc);
-        tc::tmem_ld_wait(rb);
-        if (c + 2 < kBN / kCh) {
-          tc::tmem_ld32(col0 + (c + 2) * kCh, ra);
-        } else {
-          tc::fence_before_sync();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&bars->acc_empty[b]);  // every column is in registers
-        }
-        if (kPass == 1)
-          row_chunk(rb, valid - (c + 1) * kCh, c2, ref, l);
-        else
-          col_chunk(rb, nlt + (c + 1) * kCh, c2, acc);
-        if (c + 2 < kBN / kCh) tc::tmem_ld_wait(ra);
       }
       if (kPass == 2) {
         __syncwarp();
@@ -367,13 +380,13 @@ __global__ void nl_merge_kernel(const float2* __restrict__ part, int nsplit, int
 }
 
 // Key splits for pass 1: the fewest (<= kMaxSplit) whose grid wastes at most
-// 10 % of the last wave, keeping >= 8 key tiles per split.
+// 10 % of the last wave, keeping >= 4 key tiles (1024 keys) per split.
 int choose_split(int units, int nkt) {
   const int sms = sm_count();
   int best = 1;
   double best_eff = 0.0;
   for (int s = 1; s <= kMaxSplit; ++s) {
-    if (s > 1 && nkt / s < 8) break;
+    if (s > 1 && nkt / s < 4) break;
     const double n = (double)units * s;
     const double eff = n / (ceil_div((int64_t)n, sms) * (double)sms);
     if (eff > best_eff + 1e-9) {
@@ -403,13 +416,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// [H][L][d] bf16, box = 64 elements (128 B, the swizzle span) x 128 rows x 1 head.
-bool make_map(CUtensorMap* map, const void* ptr, int H, int L, int d) {
+// [H][L][d] bf16, box = 64 elements (128 B, the swizzle span) x `rows` x 1 head.
+bool make_map(CUtensorMap* map, const void* ptr, int H, int L, int d, int rows) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)H};
   const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)L * d * 2};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -420,10 +433,13 @@ bool make_map(CUtensorMap* map, const void* ptr, int H, int L, int d) {
 template <int D>
 cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, float scale, float* imp,
                 void* ws, cudaStream_t s) {
-  CUtensorMap mq, mk;
-  if (!make_map(&mq, q, H, Lq, D) || !make_map(&mk, k, H, Lk, D)) return cudaErrorInvalidValue;
+  // A operands are 128-row tiles, B operands 256-row tiles.
+  CUtensorMap mqA, mqB, mkA, mkB;
+  if (!make_map(&mqA, q, H, Lq, D, kBM) || !make_map(&mqB, q, H, Lq, D, kBN) ||
+      !make_map(&mkA, k, H, Lk, D, kBM) || !make_map(&mkB, k, H, Lk, D, kBN))
+    return cudaErrorInvalidValue;
   int* err = reinterpret_cast<int*>(static_cast<char*>(ws) + kErrOffset);
-  const int lq_pad = (int)ceil_div(Lq, kBM) * kBM;
+  const int lq_pad = (int)ceil_div(Lq, kBN) * kBN;
   float* nl = reinterpret_cast<float*>(static_cast<char*>(ws) + kLseOffset);
   float2* part = reinterpret_cast<float2*>(
       static_cast<char*>(ws) + kLseOffset + align_up((size_t)H * lq_pad * sizeof(float), 256));
@@ -440,7 +456,7 @@ cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, float scale
   const int nkt = (int)ceil_div(Lk, kBN);
   const int nsplit = choose_split(nq * H, nkt);
   imp_tc_kernel<D, 1><<<dim3(nq * nsplit, H), kThreads, smem, s>>>(
-      mq, mk, Lq, Lk, lq_pad, nsplit, c2, nl, part, imp, err);
+      mqA, mkB, Lq, Lk, lq_pad, nsplit, c2, nl, part, imp, err);
   if (nsplit > 1) {
     const int64_t n = (int64_t)H * lq_pad;
     const int64_t blocks = ceil_div(n, 256);
@@ -448,7 +464,7 @@ cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, float scale
                                                                             lq_pad, nl);
   }
   imp_tc_kernel<D, 2><<<dim3((unsigned)ceil_div(Lk, kBM), H), kThreads, smem, s>>>(
-      mk, mq, Lq, Lk, lq_pad, 1, c2, nl, part, imp, err);
+      mkA, mqB, Lq, Lk, lq_pad, 1, c2, nl, part, imp, err);
   return cudaGetLastError();
 }
 
@@ -467,7 +483,7 @@ __global__ void exp2_selftest_kernel(const float* x, float* y_mufu, float* y_pol
 }  // namespace
 
 size_t importance_ws_bytes(int H, int Lq) {
-  const size_t rows = (size_t)H * ceil_div(Lq, kBM) * kBM;
+  const size_t rows = (size_t)H * ceil_div(Lq, kBN) * kBN;
   return kLseOffset + align_up(rows * sizeof(float), 256) + kMaxSplit * rows * sizeof(float2);
 }
 
