@@ -94,10 +94,13 @@ size_t fc_gate_workspace_size(int n_chunks, int64_t n_per_chunk);
  *              the update is not zero; 0 when both are zero)
  *   recompute  [n_chunks] uint8, out: 1 = recompute at the chunk's next
  *              forward, 0 = reuse
- *   ws         fc_gate_workspace_size() bytes.  Its first
- *              4*n_chunks bytes are completion counters that must be zero
+ *   ws         fc_gate_workspace_size() bytes.  Its first 4*(n_chunks+1)
+ *              bytes (completion counters and an error word) must be zero
  *              before the first call (e.g. cudaMemsetAsync once); every call
- *              leaves them zero again.
+ *              leaves the counters zero again.  The error word (the 32-bit
+ *              word after the n_chunks counters) becomes nonzero if a bounded
+ *              device-side wait of the streaming path gave up; the call never
+ *              clears it.
  * x and v may be NULL when n_per_chunk == 0 (then L1_rel = 0 for every
  * active chunk).
  * Errors: n_chunks < 1, n_per_chunk < 0, m < 0, null/host/misaligned
