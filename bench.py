@@ -228,29 +228,47 @@ def native(a, rank, world, local_rank):
         if world > 1:
             torch.distributed.barrier()
 
+    # One step is captured once as a CUDA graph (with timing events as graph
+    # nodes) and replayed: the GPU runs the step's launches back to back
+    # instead of waiting on the host between small kernels.
+    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
     with torch.cuda.stream(stream):
         for _ in range(a.warmup):
             flush_l2(flush, sink)
             step.run(stream)
         stream.synchronize()
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(a.steps)]
+        t0 = time.perf_counter()
+        eager_ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        flush_l2(flush, sink)
+        step.run(stream, eager_ev)
+        stream.synchronize()
+        ms_eager = eager_ev[0].elapsed_time(eager_ev[5])
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=stream, capture_error_mode="relaxed"):
+            step.run(stream, ev)
+        for _ in range(2):
+            flush_l2(flush, sink)
+            graph.replay()
+        stream.synchronize()
         clocks = Clocks(local_rank)
         barrier()
         torch.cuda.synchronize()
         clocks.start()
+        per = {n: [] for n in names}
+        tot = []
         for i in range(a.steps):
             flush_l2(flush, sink)  # between steps, outside the timed events
-            step.run(stream, evs[i])
-        stream.synchronize()
+            graph.replay()
+            stream.synchronize()
+            for j, n in enumerate(names):
+                per[n].append(ev[j].elapsed_time(ev[j + 1]))
+            tot.append(ev[0].elapsed_time(ev[5]))
         torch.cuda.synchronize()
         barrier()
         ck = clocks.stop()
-    per = {n: [] for n in names}
-    tot = []
-    for e in evs:
-        for j, n in enumerate(names):
-            per[n].append(e[j].elapsed_time(e[j + 1]))
-        tot.append(e[0].elapsed_time(e[5]))
+        gate16 = _gate_alone(W.GATE_CONFIGS["full_step_sweep"], rank, dev, stream, flush, sink,
+                             a.steps)
+    del graph
     ms_step = sum(tot) / len(tot)
     ms_call = {n: sum(v) / len(v) for n, v in per.items()}
 
@@ -291,6 +309,14 @@ def native(a, rank, world, local_rank):
                      "flops_per_launch": exec_flops, "traffic": None},
         "kernels_ms": ms_call,
         "gate": {"GB/s": gate_gbs, "frac_hbm": gate_gbs / hbm},
+        "gate_full_step_sweep": {"chunks": 16, "us": gate16 * 1e3,
+                                 "GB/s": _bytes_gate(W.GATE_CONFIGS["full_step_sweep"]) /
+                                 (gate16 * 1e-3) / 1e9,
+                                 "frac_hbm": _bytes_gate(W.GATE_CONFIGS["full_step_sweep"]) /
+                                 (gate16 * 1e-3) / 1e9 / hbm},
+        "timing": "one step captured as a CUDA graph, replayed per step; CUDA events are "
+                  "graph nodes around each call; eager (host-launched) step for reference: "
+                  f"{ms_eager:.3f} ms",
         "redundancy": {"GB/s": red_gbs, "frac_hbm": red_gbs / hbm},
         "score_topb": {"GB/s": topb_gbs},
         "compact": {"GB/s": comp_gbs, "frac_hbm": comp_gbs / hbm},
@@ -301,6 +327,39 @@ def native(a, rank, world, local_rank):
         out["e2e"] = {"value": world * Lk / (e2e["ms"] * 1e-3), "unit": UNIT,
                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
     return out
+
+
+def _gate_alone(gc, seed, dev, stream, flush, sink, steps):
+    """Gate step over every chunk of ``gc`` alone, CUDA-graph timed (ms)."""
+    import cache_gating_kv_b200 as fc
+    from cache_gating_kv_b200 import workloads as W
+
+    x = torch.from_numpy(W.gate_initial(gc, seed)).to(dev)
+    v = torch.from_numpy(W.gate_velocity(gc, seed)).to(dev)
+    st = torch.full((gc.n_chunks,), gc.m + 3, dtype=torch.int32, device=dev)
+    dt = torch.full((gc.n_chunks,), 0.001, device=dev)
+    f = torch.zeros(gc.n_chunks, device=dev)
+    l1 = torch.zeros(gc.n_chunks, device=dev)
+    mask = torch.zeros(gc.n_chunks, dtype=torch.uint8, device=dev)
+    ws = fc.workspace(fc.fc_gate_workspace_size(gc.n_chunks, gc.N), dev)
+    e0 = torch.cuda.Event(enable_timing=True, external=True)
+    e1 = torch.cuda.Event(enable_timing=True, external=True)
+    fc.fc_chunk_l1_gate(x, v, dt, st, gc.m, gc.eps[0], f, l1, mask, ws, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+        e0.record(stream)
+        fc.fc_chunk_l1_gate(x, v, dt, st, gc.m, gc.eps[0], f, l1, mask, ws, stream=stream)
+        e1.record(stream)
+    times = []
+    for i in range(steps + 3):
+        flush_l2(flush, sink)
+        g.replay()
+        stream.synchronize()
+        if i >= 3:
+            times.append(e0.elapsed_time(e1))
+    del g
+    return sum(times) / len(times)
 
 
 def _e2e(step, stream, flush, sink, a, dev):
