@@ -43,9 +43,6 @@ def flush_l2(buf, sink):
     starts with a clean L2 (no write-back traffic of ours lands on it)."""
     buf.zero_()
     torch.sum(buf.view(torch.float32), dim=0, out=sink)
-# Kernel launches per call, as implemented in cache_gating_kv_b200/csrc (importance:
-# row pass, key-split merge, column pass -- the split is taken on 148-SM B200s).
-LAUNCHES = {"gate": 1, "importance": 3, "redundancy": 1, "score_topb": 2, "compact": 1}
 
 
 def _args():
@@ -164,27 +161,35 @@ class Step:
         }
 
     def run(self, stream, ev=None):
-        """Enqueue one step; ``ev`` (6 events) brackets the five calls."""
+        """Enqueue one step; ``ev`` (6 events) brackets the five calls.
+        Returns the number of kernel launches the library enqueued."""
         fc, d, o, w = self.fc, self.d, self.out, self.ws
+        n = 0
         if ev:
             ev[0].record(stream)
         fc.fc_chunk_l1_gate(d["x"], d["vel"], d["dt"], d["step"], self.gc.m, self.eps, d["f"],
                             o["l1"], o["mask"], w["gate"], stream=stream)
+        n += fc.fc_last_launches()
         if ev:
             ev[1].record(stream)
         fc.fc_kv_importance(d["q"], d["k"], o["imp"], w["imp"], stream=stream)
+        n += fc.fc_last_launches()
         if ev:
             ev[2].record(stream)
         fc.fc_kv_redundancy(d["k"], o["red"], w["red"], stream=stream)
+        n += fc.fc_last_launches()
         if ev:
             ev[3].record(stream)
         fc.fc_kv_score_topb(o["imp"], o["red"], self.kv.pool, self.lam, self.kv.B, o["idx"],
                             w["topb"], stream=stream)
+        n += fc.fc_last_launches()
         if ev:
             ev[4].record(stream)
         fc.fc_kv_compact(d["k"], d["v"], o["idx"], o["ko"], o["vo"], stream=stream)
+        n += fc.fc_last_launches()
         if ev:
             ev[5].record(stream)
+        return n
 
     def reset_gate(self):
         self.d["x"].copy_(self.host["x"])
@@ -240,7 +245,7 @@ def native(a, rank, world, local_rank):
         t0 = time.perf_counter()
         eager_ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
         flush_l2(flush, sink)
-        step.run(stream, eager_ev)
+        launches_per_step = step.run(stream, eager_ev)
         stream.synchronize()
         ms_eager = eager_ev[0].elapsed_time(eager_ev[5])
         graph = torch.cuda.CUDAGraph()
@@ -291,7 +296,7 @@ def native(a, rank, world, local_rank):
     red_gbs = H * Lk * d * elem / (ms_call["redundancy"] * 1e-3) / 1e9
     comp_gbs = 2 * 2 * H * kv_cfg.B * d * elem / (ms_call["compact"] * 1e-3) / 1e9
     topb_gbs = H * Lk * 12 / (ms_call["score_topb"] * 1e-3) / 1e9
-    launches = sum(LAUNCHES.values()) * a.steps
+    launches = launches_per_step * a.steps
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": t_max, "higher_is_better": True, "scaling": "weak",

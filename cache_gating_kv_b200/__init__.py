@@ -22,6 +22,7 @@ __all__ = [
     "library",
     "library_path",
     "fc_version",
+    "fc_last_launches",
     "fc_chunk_l1_gate",
     "fc_chunk_l1_gate_noalloc",
     "fc_kv_importance",
@@ -57,6 +58,7 @@ def _declare(lib):
     sig = {
         "fc_last_error": (ctypes.c_char_p, []),
         "fc_version": (c_int, []),
+        "fc_last_launches": (c_int, []),
         "fc_gate_workspace_size": (c_sz, [c_int, c_i64]),
         "fc_chunk_l1_gate": (c_int, [c_p, c_p, c_int, c_i64, c_p, c_p, ctypes.c_int32, c_f, c_p,
                                      c_p, c_p, c_p, c_sz, c_p]),
@@ -126,6 +128,12 @@ def _dtype_code(t):
 
 def fc_version():
     return library().fc_version()
+
+
+def fc_last_launches():
+    """Kernel launches (memsets included) the last compute call on this thread
+    enqueued."""
+    return library().fc_last_launches()
 
 
 # ---- workspace sizes and allocation ----------------------------------------

@@ -58,6 +58,7 @@ cudaError_t run(const void* k, const void* v, int H, int Lk, const int32_t* idx,
   compact_kernel<LPR><<<grid, kCompactThreads, 0, s>>>(
       static_cast<const uint4*>(k), static_cast<const uint4*>(v), Lk, B, idx,
       static_cast<uint4*>(ko), static_cast<uint4*>(vo));
+  add_launches(1);
   return cudaGetLastError();
 }
 }  // namespace

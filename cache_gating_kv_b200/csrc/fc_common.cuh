@@ -10,6 +10,10 @@ namespace fc {
 // Device properties cached per device ordinal.
 int sm_count();
 
+// Kernel launches (and memsets) enqueued by the current C-ABI call on this
+// host thread; reported by fc_last_launches().
+void add_launches(int n);
+
 // Elements of type T packed in one 16-byte vector.
 template <typename T> struct Vec16;
 template <> struct Vec16<float> {

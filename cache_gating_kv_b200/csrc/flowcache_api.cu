@@ -24,6 +24,9 @@ int sm_count() {
   return cached[dev];
 }
 
+thread_local int g_launches = 0;
+void add_launches(int n) { g_launches += n; }
+
 }  // namespace fc
 
 namespace {
@@ -66,6 +69,7 @@ fc_status check_ptr(const void* p, const char* name) {
   } while (0)
 
 fc_status launched(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) fc::g_launches = 0;
   if (e != cudaSuccess) return fail(FC_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
   return ok();
 }
@@ -92,6 +96,8 @@ extern "C" {
 
 const char* fc_last_error(void) { return g_err; }
 
+int fc_last_launches(void) { return fc::g_launches; }
+
 int fc_version(void) { return 100; }
 
 size_t fc_gate_workspace_size(int n_chunks, int64_t n_per_chunk) {
@@ -103,6 +109,7 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
                            const float* dt, const int32_t* step, int32_t m, float eps, float* f,
                            float* l1_rel, uint8_t* recompute, void* ws, size_t ws_bytes,
                            void* stream) {
+  fc::g_launches = 0;
   if (n_chunks < 1 || n_chunks > 65535)
     return fail(FC_ERR_INVALID_ARG, "n_chunks must be in [1, 65535] (got %d)", n_chunks);
   if (n_per_chunk < 0) return fail(FC_ERR_INVALID_ARG, "n_per_chunk must be >= 0");
@@ -127,6 +134,7 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
 fc_status fc_chunk_l1_gate_noalloc(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
                                    const float* dt, const int32_t* step, int32_t m, float eps,
                                    float* f, float* l1_rel, uint8_t* recompute, void* stream) {
+  fc::g_launches = 0;
   const int max_chunks = fc::gate_noalloc_max_chunks();
   if (n_chunks < 1 || n_chunks > max_chunks)
     return fail(FC_ERR_INVALID_ARG,
@@ -159,6 +167,7 @@ size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d
 fc_status fc_kv_importance(const void* q, const void* k, fc_dtype dtype, int H, int Lq, int Lk,
                            int d, float scale, float* imp, void* ws, size_t ws_bytes,
                            void* stream) {
+  fc::g_launches = 0;
   fc_status st = check_kv_shape(dtype, H, Lq, Lk, d);
   if (st != FC_OK) return st;
   if (ws == nullptr || ws_bytes < fc::importance_ws_bytes(H, Lq))
@@ -186,6 +195,7 @@ size_t fc_redundancy_workspace_size(fc_dtype dtype, int H, int Lk, int d) {
 
 fc_status fc_kv_redundancy(const void* k, fc_dtype dtype, int H, int Lk, int d, float* red,
                            void* ws, size_t ws_bytes, void* stream) {
+  fc::g_launches = 0;
   fc_status st = check_kv_shape(dtype, H, Lk, Lk, d);
   if (st != FC_OK) return st;
   if (ws == nullptr || ws_bytes < fc::redundancy_ws_bytes(H, d))
@@ -207,6 +217,7 @@ size_t fc_score_topb_workspace_size(int H, int Lk, int B) {
 fc_status fc_kv_score_topb(const float* imp, const float* red, int H, int Lk, int pool_window,
                            float lambda, int B, float* score, int32_t* idx, void* ws,
                            size_t ws_bytes, void* stream) {
+  fc::g_launches = 0;
   if (H < 1 || H > 65535 || Lk < 1) return fail(FC_ERR_INVALID_ARG, "H and Lk must be >= 1");
   if (B < 1) return fail(FC_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
   if (pool_window < 1 || pool_window % 2 == 0 || pool_window > 511)
@@ -227,6 +238,7 @@ fc_status fc_kv_score_topb(const float* imp, const float* red, int H, int Lk, in
 
 fc_status fc_kv_compact(const void* k, const void* v, fc_dtype dtype, int H, int Lk, int d,
                         const int32_t* idx, int B, void* k_out, void* v_out, void* stream) {
+  fc::g_launches = 0;
   fc_status st = check_kv_shape(dtype, H, Lk, Lk, d);
   if (st != FC_OK) return st;
   if (B < 1) return fail(FC_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
@@ -247,6 +259,7 @@ fc_status fc_kv_compact(const void* k, const void* v, fc_dtype dtype, int H, int
 }
 
 fc_status fc_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n, void* stream) {
+  fc::g_launches = 0;
   if (n < 0 || n % 2 != 0) return fail(FC_ERR_INVALID_ARG, "n must be even and >= 0");
   if (n == 0) return ok();
   FC_CHECK_PTR(x);

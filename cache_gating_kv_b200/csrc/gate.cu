@@ -332,6 +332,7 @@ cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t N, const
     if (e != cudaSuccess) return e;
     gate_tma_kernel<<<dim3((unsigned)bpc, (unsigned)n_chunks), kTmaThreads, smem, s>>>(
         x, v, N, dt, step, m, eps, f, l1, mask, counters, partials, (int)bpc, err);
+    add_launches(1);
     return cudaGetLastError();
   }
   // Four resident 256-thread blocks per SM over the whole grid.
@@ -344,6 +345,7 @@ cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t N, const
   dim3 grid((unsigned)bpc, (unsigned)n_chunks);
   gate_kernel<<<grid, kGateThreads, 0, s>>>(x, v, N, dt, step, m, eps, f, l1, mask, counters,
                                             partials, (int)bpc);
+  add_launches(1);
   return cudaGetLastError();
 }
 
@@ -397,6 +399,7 @@ cudaError_t launch_gate_noalloc(float* x, const float* v, int n_chunks, int64_t 
   // stream first.
   e = cudaMemsetAsync(ws, 0, (size_t)(n_chunks + 1) * sizeof(unsigned), s);
   if (e != cudaSuccess) return e;
+  add_launches(1);
   return launch_gate(x, v, n_chunks, N, dt, step, m, eps, f, l1, mask, ws, s);
 }
 

@@ -185,6 +185,7 @@ cudaError_t run(const T* q, const T* k, int H, int Lq, int Lk, float scale, floa
                                                                                   c2, lse2);
   imp_col_simt<T, D><<<dim3((unsigned)ceil_div(Lk, kT), H), kThreads, smem2, s>>>(
       q, k, lse2, Lq, Lk, c2, imp);
+  add_launches(2);
   return cudaGetLastError();
 }
 }  // namespace

@@ -457,6 +457,7 @@ cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, float scale
   const int nsplit = choose_split(nq * H, nkt);
   imp_tc_kernel<D, 1><<<dim3(nq * nsplit, H), kThreads, smem, s>>>(
       mqA, mkB, Lq, Lk, lq_pad, nsplit, c2, nl, part, imp, err);
+  add_launches(nsplit > 1 ? 3 : 2);
   if (nsplit > 1) {
     const int64_t n = (int64_t)H * lq_pad;
     const int64_t blocks = ceil_div(n, 256);
@@ -498,8 +499,10 @@ cudaError_t launch_importance_tc(const void* q, const void* k, int H, int Lq, in
 cudaError_t launch_exp2_selftest(const float* x, float* y_mufu, float* y_poly, int n,
                                  cudaStream_t s) {
   const int pairs = n / 2;
-  if (pairs > 0)
+  if (pairs > 0) {
     exp2_selftest_kernel<<<(unsigned)ceil_div(pairs, 256), 256, 0, s>>>(x, y_mufu, y_poly, n);
+    add_launches(1);
+  }
   return cudaGetLastError();
 }
 

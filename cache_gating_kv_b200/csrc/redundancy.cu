@@ -68,12 +68,12 @@ __device__ __forceinline__ void load_rows(const T* kh, int r0, int hi, int sub, 
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kRedThreads)
-    red_cluster_kernel(const T* __restrict__ k, int Lk, float* __restrict__ red) {
+    red_cluster_kernel(const T* __restrict__ k, int Lk, int h0, float* __restrict__ red) {
   using L = RowLayout<T, D>;
   cg::cluster_group cluster = cg::this_cluster();
   const int nrank = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
-  const int h = blockIdx.y;
+  const int h = h0 + blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / L::LPR, cl = lane % L::LPR;
   const int per = (int)ceil_div(Lk, nrank);
@@ -182,6 +182,12 @@ __global__ void __launch_bounds__(kRedThreads)
   for (int r = lo + threadIdx.x; r < hi; r += kRedThreads) rh[r] = rh[r] * inv;
 }
 
+// Heads run in groups whose keys fit comfortably in L2 (~40 MB of K per
+// launch), so the second pass over a head's keys is served from L2 instead
+// of HBM.  Groups go from the last head to the first: the keys the importance
+// kernel touched last are the likeliest to still be cached.
+constexpr size_t kRedL2Budget = 40u << 20;
+
 template <typename T, int D>
 cudaError_t run(const T* k, int H, int Lk, float* red, cudaStream_t s) {
   // 16 CTAs per head when the slices stay long enough, else the portable 8.
@@ -191,19 +197,32 @@ cudaError_t run(const T* k, int H, int Lk, float* red, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)csize, (unsigned)H, 1);
-  cfg.blockDim = dim3(kRedThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)csize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, k, Lk, red);
+  const size_t head_bytes = (size_t)Lk * D * sizeof(T);
+  int per = (int)(kRedL2Budget / (head_bytes ? head_bytes : 1));
+  if (per < 1) per = 1;
+  if (per > H) per = H;
+  const int ngroups = (H + per - 1) / per;
+  per = (H + ngroups - 1) / ngroups;  // balance the groups
+  for (int g = ngroups - 1; g >= 0; --g) {
+    const int h0 = g * per;
+    const int nh = min(per, H - h0);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)csize, (unsigned)nh, 1);
+    cfg.blockDim = dim3(kRedThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, k, Lk, h0, red);
+    if (e != cudaSuccess) return e;
+    add_launches(1);
+  }
+  return cudaSuccess;
 }
 }  // namespace
 

@@ -16,8 +16,12 @@
 //                  the lowest indices.
 // Keys are staged in shared memory when a head's keys fit, otherwise they are
 // re-read from global memory (L2-resident) on every pass.
+#include <cooperative_groups.h>
+
 #include "fc_common.cuh"
 #include "fc_kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace fc {
 
@@ -191,6 +195,191 @@ __global__ void __launch_bounds__(kSelThreads)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Fused score + top-B for one head per thread-block cluster (the common case).
+// Each CTA of the cluster owns a contiguous slice of the head's tokens: it
+// scores its slice (pooled importance from a shared-memory tile with halo)
+// straight into shared-memory keys, every radix pass sums the CTAs' 256-bin
+// histograms through distributed shared memory (every CTA derives the same
+// digit), and the final ordered compaction offsets each CTA by the kept
+// counts of the CTAs before it.  Cluster barriers are hardware barriers.
+// ---------------------------------------------------------------------------
+constexpr int kCsThreads = 256;
+constexpr int kCsWarps = kCsThreads / 32;
+constexpr int kCsMaxSlice = 12288;  // keys per CTA held in shared memory
+
+__global__ void __launch_bounds__(kCsThreads)
+    score_select_cluster_kernel(const float* __restrict__ imp, const float* __restrict__ red,
+                                int Lk, int r, float lam, float one_minus_lam, int B,
+                                float* __restrict__ score, int32_t* __restrict__ idx) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int nrank = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int h = blockIdx.y;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int per = (int)ceil_div(Lk, nrank);
+  const int lo = min(Lk, rank * per), hi = min(Lk, lo + per);
+  const int n = hi - lo;
+
+  extern __shared__ __align__(16) unsigned char csm[];
+  uint32_t* skeys = reinterpret_cast<uint32_t*>(csm);          // [per]
+  float* tile = reinterpret_cast<float*>(csm + (size_t)per * 4);  // [per + 2r]
+  __shared__ unsigned whist[kCsWarps][256];
+  __shared__ unsigned hist[2][256];  // this CTA's histogram, double-buffered by pass
+  __shared__ unsigned s_total[256];
+  __shared__ uint32_t s_prefix, s_pmask;
+  __shared__ int s_remaining;
+  __shared__ int s_cnt[2];   // this CTA's (greater, tie) counts (read by the cluster)
+  __shared__ int s_wgt[kCsWarps], s_wtie[kCsWarps];
+
+  // ---- scores of the slice -> order-preserving keys ------------------------
+  const float* ih = imp + (size_t)h * Lk;
+  const float* rh = red + (size_t)h * Lk;
+  for (int t = tid; t < n + 2 * r; t += kCsThreads) {
+    const int j = lo - r + t;
+    tile[t] = (j >= 0 && j < Lk) ? ih[j] : -INFINITY;  // out-of-range taps ignored
+  }
+  __syncthreads();
+  for (int t = tid; t < n; t += kCsThreads) {
+    float pm = tile[t];
+    for (int o = 1; o <= 2 * r; ++o) pm = fmaxf(pm, tile[t + o]);
+    const float sc = __fsub_rn(__fmul_rn(lam, pm), __fmul_rn(one_minus_lam, rh[lo + t]));
+    if (score) score[(size_t)h * Lk + lo + t] = sc;
+    skeys[t] = order_key(sc);
+  }
+  if (tid == 0) {
+    s_prefix = 0u;
+    s_pmask = 0u;
+    s_remaining = B;
+  }
+  __syncthreads();
+
+  // ---- 4 radix passes over the cluster's keys ----------------------------------
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    const uint32_t prefix = s_prefix, pmask = s_pmask;
+    for (int i = tid; i < kCsWarps * 256; i += kCsThreads) (&whist[0][0])[i] = 0u;
+    __syncthreads();
+    for (int j0 = warp * 32; j0 < n; j0 += kCsThreads) {
+      const int j = j0 + lane;
+      uint32_t key = 0u;
+      bool in = false;
+      if (j < n) {
+        key = skeys[j];
+        in = (key & pmask) == prefix;
+      }
+      const unsigned vm = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const unsigned digit = (key >> shift) & 0xffu;
+        const unsigned peers = __match_any_sync(vm, digit);
+        if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&whist[warp][digit], __popc(peers));
+      }
+    }
+    __syncthreads();
+    {
+      unsigned t = 0u;
+#pragma unroll
+      for (int w = 0; w < kCsWarps; ++w) t += whist[w][tid];
+      hist[pass & 1][tid] = t;  // kCsThreads == 256 bins
+    }
+    cluster.sync();
+    {
+      unsigned t = 0u;
+      for (int q = 0; q < nrank; ++q) t += *cluster.map_shared_rank(&hist[pass & 1][tid], q);
+      s_total[tid] = t;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // Lane l owns bins 255-8l .. 248-8l (lane 0 the largest digits).
+      const int top = 255 - 8 * lane;
+      unsigned mine = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) mine += s_total[top - i];
+      unsigned cum = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_up_sync(0xffffffffu, cum, o);
+        if (lane >= o) cum += y;
+      }
+      const unsigned need = (unsigned)s_remaining;
+      const unsigned hit = __ballot_sync(0xffffffffu, cum >= need);
+      const int L = __ffs(hit) - 1;  // exists: the prefix holds >= need keys
+      if (lane == L) {
+        unsigned before = cum - mine;
+        int digit = top;
+        for (int i = 0; i < 8; ++i) {
+          const unsigned c = s_total[top - i];
+          if (before + c >= need) {
+            digit = top - i;
+            break;
+          }
+          before += c;
+        }
+        s_remaining = (int)(need - before);
+        s_prefix = s_prefix | ((uint32_t)digit << shift);
+        s_pmask = s_pmask | (0xffu << shift);
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- ordered compaction: keep every key > T and the first `need` keys == T ----
+  const uint32_t T = s_prefix;
+  const int need = s_remaining;
+  const int seg = (int)ceil_div(ceil_div(n, kCsWarps), 32) * 32;
+  const int w_lo = min(n, warp * seg), w_hi = min(n, w_lo + seg);
+  int gt = 0, tie = 0;
+  for (int j0 = w_lo; j0 < w_hi; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < w_hi ? skeys[j] : 0u;
+    gt += __popc(__ballot_sync(0xffffffffu, j < w_hi && key > T));
+    tie += __popc(__ballot_sync(0xffffffffu, j < w_hi && key == T));
+  }
+  if (lane == 0) {
+    s_wgt[warp] = gt;
+    s_wtie[warp] = tie;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int a = 0, b = 0;
+    for (int w = 0; w < kCsWarps; ++w) {
+      a += s_wgt[w];
+      b += s_wtie[w];
+    }
+    s_cnt[0] = a;
+    s_cnt[1] = b;
+  }
+  cluster.sync();
+  // Counts of the CTAs before this one (their tokens come first).
+  int gt_base = 0, tie_base = 0;
+  for (int q = 0; q < rank; ++q) {
+    gt_base += *cluster.map_shared_rank(&s_cnt[0], q);
+    tie_base += *cluster.map_shared_rank(&s_cnt[1], q);
+  }
+  for (int w = 0; w < warp; ++w) {
+    gt_base += s_wgt[w];
+    tie_base += s_wtie[w];
+  }
+  int out = gt_base + min(need, tie_base);
+  int tie_run = tie_base;
+  const unsigned lt = (1u << lane) - 1u;
+  int32_t* oh = idx + (size_t)h * B;
+  for (int j0 = w_lo; j0 < w_hi; j0 += 32) {
+    const int j = j0 + lane;
+    const uint32_t key = j < w_hi ? skeys[j] : 0u;
+    const bool is_gt = j < w_hi && key > T;
+    const bool is_tie = j < w_hi && key == T;
+    const unsigned tb = __ballot_sync(0xffffffffu, is_tie);
+    const bool sel = is_gt || (is_tie && tie_run + __popc(tb & lt) < need);
+    const unsigned sb = __ballot_sync(0xffffffffu, sel);
+    const int pos = out + __popc(sb & lt);
+    if (sel && pos < B) oh[pos] = lo + j;  // pos < B always holds; the check keeps writes in bounds
+    out += __popc(sb);
+    tie_run += __popc(tb);
+  }
+  cluster.sync();  // no CTA leaves while another may still read its shared memory
+}
+
 __global__ void fill_all_kernel(int32_t* idx, int Lk, int B, int H) {
   const int64_t n = (int64_t)H * B;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
@@ -208,9 +397,40 @@ cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk,
                               cudaStream_t s) {
   uint32_t* keys = static_cast<uint32_t*>(ws);
   const float one_minus = 1.0f - lambda;  // float32, as the score's definition
+  const int r = pool / 2;
+  if (B < Lk && Lk <= 16 * kCsMaxSlice) {
+    // One cluster per head: 8 CTAs, or 16 (non-portable) for long histories.
+    const int csize = Lk > 8 * 4096 ? 16 : 8;
+    const int per = (int)ceil_div(Lk, csize);
+    const size_t smem = (size_t)per * 4 + (size_t)(per + 2 * r) * 4;
+    auto kern = score_select_cluster_kernel;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    if (csize > 8) {
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)csize, (unsigned)H, 1);
+    cfg.blockDim = dim3(kCsThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, imp, red, Lk, r, lambda, one_minus, B, score, idx);
+    if (e != cudaSuccess) return e;
+    add_launches(1);
+    return cudaSuccess;
+  }
   dim3 g1((unsigned)ceil_div(Lk, kScoreTile), H);
-  score_kernel<<<g1, kScoreThreads, 0, s>>>(imp, red, Lk, pool / 2, lambda, one_minus, score,
-                                            keys);
+  score_kernel<<<g1, kScoreThreads, 0, s>>>(imp, red, Lk, r, lambda, one_minus, score, keys);
+  add_launches(2);  // the score kernel and one selection (or keep-all) kernel
   if (B >= Lk) {
     const int64_t nfb = ceil_div((int64_t)H * B, 256);
     fill_all_kernel<<<(unsigned)(nfb < 1024 ? nfb : 1024), 256, 0, s>>>(

@@ -58,6 +58,10 @@ const char* fc_last_error(void);
 /* Library version, as major*10000 + minor*100 + patch. */
 int fc_version(void);
 
+/* Kernel launches (memsets included) that the last compute call made on this
+ * host thread enqueued; 0 after an error.  For accounting in benchmarks. */
+int fc_last_launches(void);
+
 /* ------------------------------------------------------------------------ */
 /* Chunkwise cache gate (key design 1: relative L1 distance; key design 2:  */
 /* the accumulator f)                                                       */
