@@ -20,7 +20,8 @@
 //   3. every CTA scales its rows by 1/sum_j e_j.
 // The cluster barriers are hardware barriers (no spin loops).  Each 16-byte
 // lane vector holds 8 bf16 or 4 fp32 elements; a row is d*elem/16 lanes of a
-// warp, and every lane keeps four rows' loads in flight.
+// warp, and every lane keeps eight rows' loads in flight (a CTA ~32 KB, three
+// CTAs per SM).
 #include <cooperative_groups.h>
 
 #include "fc_common.cuh"
@@ -33,7 +34,7 @@ namespace fc {
 namespace {
 constexpr int kRedThreads = 256;
 constexpr int kRedWarps = kRedThreads / 32;
-constexpr int kRedUnroll = 4;
+constexpr int kRedUnroll = 8;  // 16-byte loads in flight per lane
 
 template <typename T, int D>
 struct RowLayout {
@@ -54,16 +55,13 @@ __device__ __forceinline__ float row_sum(float v) {
 
 template <typename T, int D>
 __device__ __forceinline__ void load_rows(const T* kh, int r0, int hi, int sub, int cl,
-                                          float (&e)[kRedUnroll][RowLayout<T, D>::EPL]) {
+                                          uint4 (&u)[kRedUnroll]) {
   using L = RowLayout<T, D>;
-  uint4 u[kRedUnroll];
 #pragma unroll
   for (int i = 0; i < kRedUnroll; ++i) {
     const int r = r0 + i * L::RPW + sub;
     u[i] = r < hi ? ld_nc_v4(kh + (size_t)r * D + cl * L::EPL) : make_uint4(0u, 0u, 0u, 0u);
   }
-#pragma unroll
-  for (int i = 0; i < kRedUnroll; ++i) Vec16<T>::to_float(u[i], e[i]);
 }
 
 template <typename T, int D>
@@ -93,17 +91,19 @@ __global__ void __launch_bounds__(kRedThreads)
 #pragma unroll
   for (int i = 0; i < L::EPL; ++i) acc[i] = 0.0f;
   for (int r0 = lo + warp * L::RPW * kRedUnroll; r0 < hi; r0 += kRowsPerIter) {
-    float e[kRedUnroll][L::EPL];
-    load_rows<T, D>(kh, r0, hi, sub, cl, e);
+    uint4 raw[kRedUnroll];
+    load_rows<T, D>(kh, r0, hi, sub, cl, raw);
 #pragma unroll
     for (int u = 0; u < kRedUnroll; ++u) {
+      float e[L::EPL];
+      Vec16<T>::to_float(raw[u], e);
       float n2 = 0.0f;
 #pragma unroll
-      for (int i = 0; i < L::EPL; ++i) n2 = fmaf(e[u][i], e[u][i], n2);
+      for (int i = 0; i < L::EPL; ++i) n2 = fmaf(e[i], e[i], n2);
       n2 = row_sum<L::LPR>(n2);
       const float inv = 1.0f / fmaxf(sqrtf(n2), 1e-12f);  // a zero key stays zero
 #pragma unroll
-      for (int i = 0; i < L::EPL; ++i) acc[i] = fmaf(e[u][i], inv, acc[i]);
+      for (int i = 0; i < L::EPL; ++i) acc[i] = fmaf(e[i], inv, acc[i]);
     }
   }
 #pragma unroll
@@ -137,15 +137,17 @@ __global__ void __launch_bounds__(kRedThreads)
   float* rh = red + (size_t)h * Lk;
   double esum = 0.0;
   for (int r0 = lo + warp * L::RPW * kRedUnroll; r0 < hi; r0 += kRowsPerIter) {
-    float e[kRedUnroll][L::EPL];
-    load_rows<T, D>(kh, r0, hi, sub, cl, e);
+    uint4 raw[kRedUnroll];
+    load_rows<T, D>(kh, r0, hi, sub, cl, raw);
 #pragma unroll
     for (int u = 0; u < kRedUnroll; ++u) {
+      float e[L::EPL];
+      Vec16<T>::to_float(raw[u], e);
       float n2 = 0.0f, dot = 0.0f;
 #pragma unroll
       for (int i = 0; i < L::EPL; ++i) {
-        n2 = fmaf(e[u][i], e[u][i], n2);
-        dot = fmaf(e[u][i], sv[i], dot);
+        n2 = fmaf(e[i], e[i], n2);
+        dot = fmaf(e[i], sv[i], dot);
       }
       n2 = row_sum<L::LPR>(n2);
       dot = row_sum<L::LPR>(dot);
@@ -182,12 +184,6 @@ __global__ void __launch_bounds__(kRedThreads)
   for (int r = lo + threadIdx.x; r < hi; r += kRedThreads) rh[r] = rh[r] * inv;
 }
 
-// Heads run in groups whose keys fit comfortably in L2 (~40 MB of K per
-// launch), so the second pass over a head's keys is served from L2 instead
-// of HBM.  Groups go from the last head to the first: the keys the importance
-// kernel touched last are the likeliest to still be cached.
-constexpr size_t kRedL2Budget = 40u << 20;
-
 template <typename T, int D>
 cudaError_t run(const T* k, int H, int Lk, float* red, cudaStream_t s) {
   // 16 CTAs per head when the slices stay long enough, else the portable 8.
@@ -197,31 +193,21 @@ cudaError_t run(const T* k, int H, int Lk, float* red, cudaStream_t s) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
   }
-  const size_t head_bytes = (size_t)Lk * D * sizeof(T);
-  int per = (int)(kRedL2Budget / (head_bytes ? head_bytes : 1));
-  if (per < 1) per = 1;
-  if (per > H) per = H;
-  const int ngroups = (H + per - 1) / per;
-  per = (H + ngroups - 1) / ngroups;  // balance the groups
-  for (int g = ngroups - 1; g >= 0; --g) {
-    const int h0 = g * per;
-    const int nh = min(per, H - h0);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)csize, (unsigned)nh, 1);
-    cfg.blockDim = dim3(kRedThreads, 1, 1);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)csize;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, k, Lk, h0, red);
-    if (e != cudaSuccess) return e;
-    add_launches(1);
-  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)csize, (unsigned)H, 1);
+  cfg.blockDim = dim3(kRedThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, k, Lk, 0, red);
+  if (e != cudaSuccess) return e;
+  add_launches(1);
   return cudaSuccess;
 }
 }  // namespace
