@@ -14,14 +14,16 @@
 //   1. every CTA sums khat over its rows; the partial d-vectors are exchanged
 //      through distributed shared memory and every CTA adds them in rank order
 //      (identical s everywhere, deterministic);
-//   2. every CTA re-reads its rows (now L2-resident), forms r_j and
+//   2. every CTA re-reads its rows backwards (the last ones read are still in
+//      L2), forms r_j and
 //      e_j = exp(r_j), writes e_j, and the per-CTA sums of e_j are exchanged
 //      the same way;
 //   3. every CTA scales its rows by 1/sum_j e_j.
-// The cluster barriers are hardware barriers (no spin loops).  Each 16-byte
-// lane vector holds 8 bf16 or 4 fp32 elements; a row is d*elem/16 lanes of a
-// warp, and every lane keeps eight rows' loads in flight (a CTA ~32 KB, three
-// CTAs per SM).
+// The cluster barriers are hardware barriers (no spin loops).  Each lane
+// holds two 16-byte vectors of a row (16 bf16 or 8 fp32 elements), so a row's
+// reductions take log2(d*elem/32) shuffles; the per-row scalars use the
+// special-function unit (rsqrt, ex2: ~2^-22 relative error); every lane keeps
+// four rows' loads in flight.
 #include <cooperative_groups.h>
 
 #include "fc_common.cuh"
@@ -34,15 +36,27 @@ namespace fc {
 namespace {
 constexpr int kRedThreads = 256;
 constexpr int kRedWarps = kRedThreads / 32;
-constexpr int kRedUnroll = 8;  // 16-byte loads in flight per lane
+constexpr int kRedUnroll = 2;  // rows in flight per lane (two 16-byte loads each)
 
+// Each lane holds two 16-byte vectors (32 contiguous bytes) of a row.
 template <typename T, int D>
 struct RowLayout {
-  static constexpr int EPL = Vec16<T>::N;  // elements per lane
-  static constexpr int LPR = D / EPL;      // lanes per row
-  static constexpr int RPW = 32 / LPR;     // rows per warp step
+  static constexpr int VPL = 2;                     // vectors per lane
+  static constexpr int EPL = VPL * Vec16<T>::N;     // elements per lane
+  static constexpr int LPR = D / EPL;               // lanes per row
+  static constexpr int RPW = 32 / LPR;              // rows per warp step
   static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "row layout");
 };
+
+// 1/max(||k||, 1e-12) from ||k||^2 on the special-function unit.
+__device__ __forceinline__ float inv_norm(float n2) {
+  return n2 > 1e-24f ? rsqrtf(n2) : 1e12f;
+}
+__device__ __forceinline__ float exp_fast(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x * 1.4426950408889634f));
+  return y;
+}
 
 // Sum over the LPR lanes that hold one row (xor offsets below LPR stay inside
 // the row's lane group).
@@ -55,13 +69,21 @@ __device__ __forceinline__ float row_sum(float v) {
 
 template <typename T, int D>
 __device__ __forceinline__ void load_rows(const T* kh, int r0, int hi, int sub, int cl,
-                                          uint4 (&u)[kRedUnroll]) {
+                                          uint4 (&u)[kRedUnroll][2]) {
   using L = RowLayout<T, D>;
 #pragma unroll
   for (int i = 0; i < kRedUnroll; ++i) {
     const int r = r0 + i * L::RPW + sub;
-    u[i] = r < hi ? ld_nc_v4(kh + (size_t)r * D + cl * L::EPL) : make_uint4(0u, 0u, 0u, 0u);
+    const T* p = kh + (size_t)r * D + cl * L::EPL;
+    u[i][0] = r < hi ? ld_nc_v4(p) : make_uint4(0u, 0u, 0u, 0u);
+    u[i][1] = r < hi ? ld_nc_v4(p + Vec16<T>::N) : make_uint4(0u, 0u, 0u, 0u);
   }
+}
+
+template <typename T, int D>
+__device__ __forceinline__ void unpack(const uint4 (&u)[2], float* e) {
+  Vec16<T>::to_float(u[0], e);
+  Vec16<T>::to_float(u[1], e + Vec16<T>::N);
 }
 
 template <typename T, int D>
@@ -91,17 +113,17 @@ __global__ void __launch_bounds__(kRedThreads)
 #pragma unroll
   for (int i = 0; i < L::EPL; ++i) acc[i] = 0.0f;
   for (int r0 = lo + warp * L::RPW * kRedUnroll; r0 < hi; r0 += kRowsPerIter) {
-    uint4 raw[kRedUnroll];
+    uint4 raw[kRedUnroll][2];
     load_rows<T, D>(kh, r0, hi, sub, cl, raw);
 #pragma unroll
     for (int u = 0; u < kRedUnroll; ++u) {
       float e[L::EPL];
-      Vec16<T>::to_float(raw[u], e);
+      unpack<T, D>(raw[u], e);
       float n2 = 0.0f;
 #pragma unroll
       for (int i = 0; i < L::EPL; ++i) n2 = fmaf(e[i], e[i], n2);
       n2 = row_sum<L::LPR>(n2);
-      const float inv = 1.0f / fmaxf(sqrtf(n2), 1e-12f);  // a zero key stays zero
+      const float inv = inv_norm(n2);  // a zero key stays zero
 #pragma unroll
       for (int i = 0; i < L::EPL; ++i) acc[i] = fmaf(e[i], inv, acc[i]);
     }
@@ -136,13 +158,17 @@ __global__ void __launch_bounds__(kRedThreads)
   const float inv_lk = 1.0f / (float)Lk;
   float* rh = red + (size_t)h * Lk;
   double esum = 0.0;
-  for (int r0 = lo + warp * L::RPW * kRedUnroll; r0 < hi; r0 += kRowsPerIter) {
-    uint4 raw[kRedUnroll];
+  // Backwards over the slice: the rows read last by step 1 come first, while
+  // they are still in L2.
+  const int n_iter = (int)ceil_div(hi - lo, kRowsPerIter);
+  for (int it = n_iter - 1; it >= 0; --it) {
+    const int r0 = lo + it * kRowsPerIter + warp * L::RPW * kRedUnroll;
+    uint4 raw[kRedUnroll][2];
     load_rows<T, D>(kh, r0, hi, sub, cl, raw);
 #pragma unroll
     for (int u = 0; u < kRedUnroll; ++u) {
       float e[L::EPL];
-      Vec16<T>::to_float(raw[u], e);
+      unpack<T, D>(raw[u], e);
       float n2 = 0.0f, dot = 0.0f;
 #pragma unroll
       for (int i = 0; i < L::EPL; ++i) {
@@ -151,10 +177,10 @@ __global__ void __launch_bounds__(kRedThreads)
       }
       n2 = row_sum<L::LPR>(n2);
       dot = row_sum<L::LPR>(dot);
-      const float inv = 1.0f / fmaxf(sqrtf(n2), 1e-12f);
+      const float inv = inv_norm(n2);
       // r_j = (khat_j . s - ||khat_j||^2) / L_k
       const float rj = (dot * inv - n2 * inv * inv) * inv_lk;
-      const float ej = expf(rj);
+      const float ej = exp_fast(rj);
       const int r = r0 + u * L::RPW + sub;
       if (r < hi && cl == 0) {
         rh[r] = ej;
