@@ -311,7 +311,11 @@ def native(a, rank, world, local_rank):
         "roofline": {"bound": "tensor", "kernel": "fc_kv_importance (2 passes)",
                      "achieved": imp_tf, "peak": tf_burst, "unit": "TFLOP/s",
                      "frac": imp_tf / tf_burst, "peak_source": f"{src} bf16 burst",
-                     "flops_per_launch": exec_flops, "traffic": None},
+                     "flops_per_launch": exec_flops,
+                     # DRAM read + write of the call's three launches, from the ncu capture
+                     # of this kernel version (profiles/step_kernels_bf16_layer.md)
+                     "traffic": 263.2e6 if a.workload == "bf16_layer" else None,
+                     "traffic_unit": "bytes per call"},
         "kernels_ms": ms_call,
         "gate": {"GB/s": gate_gbs, "frac_hbm": gate_gbs / hbm},
         "gate_full_step_sweep": {"chunks": 16, "us": gate16 * 1e3,
