@@ -27,6 +27,8 @@ size_t importance_ws_bytes(int H, int Lq);
 cudaError_t launch_importance_tc(const void* q, const void* k, int H, int Lq, int Lk, int d,
                                  float scale, float* imp, void* ws, cudaStream_t s);
 bool importance_tc_supported(int d);
+// A bounded mbarrier wait that nothing completes, for the self-test
+cudaError_t launch_wait_selftest(long long limit_cycles, int* err, cudaStream_t s);
 // 2^x on the special-function unit and on the FMA pipes, for the self-test
 cudaError_t launch_exp2_selftest(const float* x, float* y_mufu, float* y_poly, int n,
                                  cudaStream_t s);

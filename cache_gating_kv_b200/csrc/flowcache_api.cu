@@ -269,4 +269,13 @@ fc_status fc_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n, 
                   "fc_selftest_exp2");
 }
 
+fc_status fc_selftest_wait_timeout(long long limit_cycles, int* err, void* stream) {
+  fc::g_launches = 0;
+  if (limit_cycles < 0 || limit_cycles > 4000000000ll)
+    return fail(FC_ERR_INVALID_ARG, "limit_cycles must be in [0, 4e9]");
+  FC_CHECK_PTR(err);
+  return launched(fc::launch_wait_selftest(limit_cycles, err, static_cast<cudaStream_t>(stream)),
+                  "fc_selftest_wait_timeout");
+}
+
 }  // extern "C"

@@ -481,7 +481,26 @@ __global__ void exp2_selftest_kernel(const float* x, float* y_mufu, float* y_pol
     y_poly[i + 1] = p.y;
   }
 }
+// Self-test of the bounded wait: every thread waits on an mbarrier that
+// nothing arrives on, gives up after `limit` clocks and records it.
+__global__ void wait_selftest_kernel(long long limit, int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::fence_barrier_init();
+  }
+  __syncthreads();
+  const bool ok = tc::mbar_wait(&bar, 0, limit);
+  if (!ok && threadIdx.x == 0) atomicAdd(err, 1);
+  __syncthreads();
+}
 }  // namespace
+
+cudaError_t launch_wait_selftest(long long limit_cycles, int* err, cudaStream_t s) {
+  wait_selftest_kernel<<<1, 32, 0, s>>>(limit_cycles, err);
+  add_launches(1);
+  return cudaGetLastError();
+}
 
 size_t importance_ws_bytes(int H, int Lq) {
   const size_t rows = (size_t)H * ceil_div(Lq, kBN) * kBN;

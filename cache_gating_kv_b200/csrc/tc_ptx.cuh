@@ -45,12 +45,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0;
 }
 // Wait for the phase of parity `parity` to complete; false if it did not
-// within kWaitCycles (the caller records the error and winds down).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// within `limit` SM clocks (the caller records the error and winds down).
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          long long limit = kWaitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
-    if (clock64() - t0 > kWaitCycles) return false;
+    if (clock64() - t0 > limit) return false;
   }
   return true;
 }

@@ -18,6 +18,8 @@ that any head of any layer can be drawn on its own.  bf16 workloads round Q, K
 and V to bfloat16 once; both sides consume those rounded values.
 """
 
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 from typing import Optional, Sequence, Tuple
 
@@ -127,10 +129,12 @@ def _rng(seed, role, layer=0, head=0):
 
 
 def _ar1(rng, L, d, rho, noise):
-    """AR(1) walk along tokens: x_0 ~ N(0,I), x_j = rho*x_{j-1} + noise*n_j."""
+    """AR(1) walk along tokens: x_0 ~ N(0,I), x_j = rho*x_{j-1} + noise*n_j.
+    Returns a C-contiguous float64 [L, d] array."""
     n = rng.standard_normal((d, L), dtype=np.float32).astype(np.float64)
     n[:, 0] /= noise  # so that the filter's first output is n_0 itself
-    return scipy.signal.lfilter([noise], [1.0, -rho], n, axis=1).T
+    y = scipy.signal.lfilter([noise], [1.0, -rho], n, axis=1)
+    return torch.from_numpy(y).t().contiguous().numpy()
 
 
 def _keys_one_head(cfg: KVConfig, seed, layer, head):
@@ -186,22 +190,30 @@ def kv_head(cfg: KVConfig, seed=0, layer=0, head=0):
 
 
 def _round_bf16(a):
-    return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).float().numpy()
+    return torch.from_numpy(a).to(torch.bfloat16).float().numpy()
 
 
 def kv_inputs(cfg: KVConfig, seed=0, layer=0, heads: Optional[Sequence[int]] = None):
     """Q [H,L_q,d], K [H,L_k,d], V [H,L_k,d] as torch CPU tensors in the
     workload's dtype (torch.bfloat16 or torch.float32).  ``heads`` selects a
     subset (default: all heads)."""
-    heads = range(cfg.H) if heads is None else heads
+    heads = list(range(cfg.H)) if heads is None else list(heads)
     tdt = torch.bfloat16 if cfg.dtype == "bf16" else torch.float32
-    qs, ks, vs = [], [], []
-    for h in heads:
-        q, k, v = kv_head(cfg, seed, layer, h)
-        qs.append(torch.from_numpy(q).to(tdt))
-        ks.append(torch.from_numpy(k).to(tdt))
-        vs.append(torch.from_numpy(v).to(tdt))
-    return torch.stack(qs), torch.stack(ks), torch.stack(vs)
+    Q = torch.empty(len(heads), cfg.Lq, cfg.d, dtype=tdt)
+    K = torch.empty(len(heads), cfg.Lk, cfg.d, dtype=tdt)
+    V = torch.empty(len(heads), cfg.Lk, cfg.d, dtype=tdt)
+
+    def one(i):
+        q, k, v = kv_head(cfg, seed, layer, heads[i])
+        Q[i] = torch.from_numpy(q)
+        K[i] = torch.from_numpy(k)
+        V[i] = torch.from_numpy(v)
+
+    # heads are independent streams: draw them on a few threads
+    workers = max(1, min(len(heads), (os.cpu_count() or 2) // 2, 8))
+    with ThreadPoolExecutor(workers) as ex:
+        list(ex.map(one, range(len(heads))))
+    return Q, K, V
 
 
 # ---------------------------------------------------------------------------

@@ -23,6 +23,15 @@ extern "C" {
  */
 fc_status fc_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n, void* stream);
 
+/*
+ * Failure-path self-test of the bounded device-side waits the tensor-core and
+ * streaming kernels use: one CTA waits on an mbarrier that nothing arrives on,
+ * gives up after `limit_cycles` SM clocks, and adds 1 to *err (a device int
+ * the caller zeroes).  The kernel then returns normally: the context stays
+ * usable.  limit_cycles in [0, 4e9] (4e9 ~ 2 s at 1.9 GHz).
+ */
+fc_status fc_selftest_wait_timeout(long long limit_cycles, int* err, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

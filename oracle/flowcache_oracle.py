@@ -46,6 +46,7 @@ import numpy as np
 
 __all__ = [
     "gate_step",
+    "history_gate_step",
     "importance",
     "row_lse",
     "importance_at",
@@ -119,6 +120,54 @@ def gate_step(x, v, dt, step, m, eps, f):
                 mask[c] = 0  # reuse and accumulate
                 f_next[c] = acc
     return x_next, f_next, l1, mask
+
+
+def history_gate_step(h_old, h_new, step, m, delta, f):
+    """One step of the history-guided cache gate (a neighbouring method: the
+    ARCache notes "Accelerating Autoregressive Video Diffusion via
+    History-Guided Cache and Residual Correction", 关键设计 1, HGC).
+
+    Delta = ||h_t - h_{t+1}||_1 / ||h_{t+1}||_1 (denominator at the older step
+    h_{t+1}); the deviations are summed from the last refresh step t_ref down
+    to t, and the step where the sum first exceeds delta refreshes:
+    sum_{i=t+1}^{t_ref} Delta <= delta < sum_{i=t}^{t_ref} Delta.  The refresh
+    step becomes t_ref, so its own Delta opens the next window (f = Delta after
+    a refresh, where the FlowCache gate resets to 0).  The first m steps of a
+    segment refresh unconditionally (same rule for f).
+
+    h_old [n, N] float32 h_{t+1}; h_new [n, N] float32 h_t; step [n] (< 0:
+    inactive, untouched); f [n] float32.  Returns (h_next = h_new copy for
+    active segments, f_next, d_rel, refresh mask)."""
+    h_old = np.asarray(h_old, dtype=np.float32)
+    h_new = np.asarray(h_new, dtype=np.float32)
+    step = np.asarray(step)
+    f = np.asarray(f, dtype=np.float32)
+    n = h_old.shape[0]
+    delta32 = np.float32(delta)
+    h_next = h_old.copy()
+    f_next = f.copy()
+    d = np.zeros(n, dtype=np.float32)
+    mask = np.zeros(n, dtype=np.uint8)
+    for c in range(n):
+        if step[c] < 0:
+            continue
+        diff = h_new[c] - h_old[c]  # one float32 rounding
+        num = np.sum(np.abs(diff.astype(np.float64)))
+        den = np.sum(np.abs(h_old[c].astype(np.float64)))
+        if den > 0.0:
+            rel = num / den
+        else:
+            rel = math.inf if num > 0.0 else 0.0
+        d[c] = np.float32(rel)
+        h_next[c] = h_new[c]
+        acc = np.float32(f[c] + d[c])
+        if step[c] < m or acc > delta32:
+            mask[c] = 1
+            f_next[c] = d[c]  # the refresh step opens the next window
+        else:
+            mask[c] = 0
+            f_next[c] = acc
+    return h_next, f_next, d, mask
 
 
 # ---------------------------------------------------------------------------

@@ -116,3 +116,16 @@ def test_product_package_does_not_import_the_oracle():
         src = open(path, errors="replace").read()
         assert not re.search(r"^\s*(import|from)\s+oracle\b", src, re.M), path
         assert "flowcache_oracle" not in src, path
+
+
+def test_selftest_entries_validate_on_the_host():
+    import ctypes as C
+    lib = fc.library()
+    lib.fc_selftest_wait_timeout.restype = C.c_int
+    lib.fc_selftest_wait_timeout.argtypes = [C.c_longlong, C.c_void_p, C.c_void_p]
+    assert lib.fc_selftest_wait_timeout(-1, None, None) == 1
+    assert lib.fc_selftest_wait_timeout(10**10, None, None) == 1
+    assert lib.fc_selftest_wait_timeout(1000, None, None) == 1  # NULL error word
+    lib.fc_selftest_exp2.restype = C.c_int
+    lib.fc_selftest_exp2.argtypes = [C.c_void_p] * 3 + [C.c_int, C.c_void_p]
+    assert lib.fc_selftest_exp2(None, None, None, 3, None) == 1  # odd n

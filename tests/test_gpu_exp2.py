@@ -48,3 +48,20 @@ def test_polynomial_exp2_clamps_below():
     ym, yp = _run(x)
     assert np.all(ym[:3] == 0)
     np.testing.assert_allclose(yp, 2.0 ** -125, rtol=3e-7)
+
+
+def test_bounded_wait_gives_up_and_context_stays_usable():
+    """A wait on an mbarrier nothing arrives on returns after its limit and
+    records an error word; the context keeps working afterwards."""
+    lib = fc.library()
+    lib.fc_selftest_wait_timeout.restype = ctypes.c_int
+    lib.fc_selftest_wait_timeout.argtypes = [ctypes.c_longlong, ctypes.c_void_p, ctypes.c_void_p]
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    st = lib.fc_selftest_wait_timeout(2_000_000, err.data_ptr(),
+                                      torch.cuda.current_stream().cuda_stream)
+    assert st == 0, lib.fc_last_error()
+    torch.cuda.synchronize()
+    assert int(err.item()) == 1
+    # the device is still usable: a regular library call succeeds
+    ym, yp = _run(np.array([0.0, 1.0], np.float32))
+    assert ym[1] == 2.0 and abs(yp[1] - 2.0) < 1e-6

@@ -375,3 +375,59 @@ def test_compact_is_a_gather():
         np.testing.assert_array_equal(ko[h][idx[h] >= 0], kt[h].index_select(0, sel)[idx[h] >= 0])
     assert np.all(ko[0, 3] == 0) and np.all(vo[0, 3] == 0)
     np.testing.assert_array_equal(vo[1], v[1, 1:5])
+
+
+# ---------------------------------------------------------------------------
+# History-guided gate (the neighbouring ARCache method's HGC rule)
+# ---------------------------------------------------------------------------
+def test_history_gate_hand_trace(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "history_gate_trace.json")))
+    N = g["N"]
+    f = np.zeros(1, np.float32)
+    for t in range(g["steps"]):
+        h_old = np.full((1, N), g["h_old"], np.float32)
+        h_new = np.full((1, N), g["h_new"], np.float32)
+        h_next, f, d, mask = O.history_gate_step(h_old, h_new, np.int32([t]), g["m"], g["delta"], f)
+        assert d[0] == np.float32(g["d"])
+        assert mask[0] == g["mask"][t], t
+        assert f[0] == np.float32(g["f"][t]), t
+        assert np.all(h_next == np.float32(g["h_new"]))
+
+
+def test_history_gate_denominator_is_the_older_step():
+    """h_old = 2, h_new = 3: Delta = 1/2 (older step in the denominator), not 1/3."""
+    h_old = np.full((1, 64), 2.0, np.float32)
+    h_new = np.full((1, 64), 3.0, np.float32)
+    _, _, d, _ = O.history_gate_step(h_old, h_new, np.int32([5]), 0, 10.0, np.zeros(1, np.float32))
+    assert d[0] == np.float32(0.5)
+
+
+def test_history_gate_matches_cumulative_rule_brute_force():
+    """Random Delta sequences: the refresh steps are exactly those where the
+    window sum from the last refresh (inclusive) first exceeds delta."""
+    rng = np.random.default_rng(13)
+    for trial in range(20):
+        deltas = rng.uniform(0.0, 0.04, size=25).astype(np.float32)
+        thr = float(rng.uniform(0.02, 0.1))
+        f = np.zeros(1, np.float32)
+        got = []
+        for t, dv in enumerate(deltas):
+            h_old = np.ones((1, 256), np.float32)
+            h_new = h_old + np.float32(dv)
+            # the Delta the gate sees is the float32 value of (h_new - 1) on each element
+            _, f, d, mask = O.history_gate_step(h_old, h_new, np.int32([t]), 0, thr, f)
+            got.append((int(mask[0]), float(d[0])))
+        # brute force on the observed Deltas: window sums from t_ref, inclusive
+        ds = [dd for _, dd in got]
+        exp, window = [], []
+        for t, dd in enumerate(ds):
+            window.append(dd)
+            s = np.float32(0.0)
+            for w in window:
+                s = np.float32(s + np.float32(w))
+            if s > np.float32(thr):
+                exp.append(1)
+                window = [dd]
+            else:
+                exp.append(0)
+        assert [m for m, _ in got] == exp
