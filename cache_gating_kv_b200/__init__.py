@@ -25,6 +25,7 @@ __all__ = [
     "fc_last_launches",
     "fc_chunk_l1_gate",
     "fc_chunk_l1_gate_noalloc",
+    "fc_history_l1_gate",
     "fc_kv_importance",
     "fc_kv_redundancy",
     "fc_kv_score_topb",
@@ -64,6 +65,8 @@ def _declare(lib):
                                      c_p, c_p, c_p, c_sz, c_p]),
         "fc_chunk_l1_gate_noalloc": (c_int, [c_p, c_p, c_int, c_i64, c_p, c_p, ctypes.c_int32,
                                              c_f, c_p, c_p, c_p, c_p]),
+        "fc_history_l1_gate": (c_int, [c_p, c_p, c_int, c_i64, c_p, ctypes.c_int32, c_f, c_p, c_p,
+                                       c_p, c_p, c_sz, c_p]),
         "fc_importance_workspace_size": (c_sz, [c_int, c_int, c_int, c_int, c_int]),
         "fc_kv_importance": (c_int, [c_p, c_p, c_int, c_int, c_int, c_int, c_int, c_f, c_p, c_p,
                                      c_sz, c_p]),
@@ -168,6 +171,17 @@ def fc_chunk_l1_gate(x, v, dt, step, m, eps, f, l1_rel, recompute, ws, stream=No
                                      _p(f), _p(l1_rel), _p(recompute), _p(ws), ws.numel(),
                                      _s(stream))
     _check("fc_chunk_l1_gate", st)
+
+
+def fc_history_l1_gate(h_old, h_new, step, m, delta, f, d_rel, refresh, ws, stream=None):
+    """History-guided gate step (in place on ``h_old`` and ``f``): h_old is
+    h_{t+1} in and h_t out.  [n, N] float32 snapshots; step [n] int32; f, d_rel
+    [n] float32; refresh [n] uint8; ws from :func:`fc_gate_workspace_size`."""
+    n, N = h_old.shape
+    st = library().fc_history_l1_gate(_p(h_old), _p(h_new), n, N, _p(step), int(m), float(delta),
+                                       _p(f), _p(d_rel), _p(refresh), _p(ws), ws.numel(),
+                                       _s(stream))
+    _check("fc_history_l1_gate", st)
 
 
 def fc_chunk_l1_gate_noalloc(x, v, dt, step, m, eps, f, l1_rel, recompute, stream=None):

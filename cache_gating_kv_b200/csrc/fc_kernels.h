@@ -10,9 +10,11 @@ namespace fc {
 
 // ---- chunkwise gate --------------------------------------------------------
 size_t gate_ws_bytes(int n_chunks);
+// history = false: FlowCache (x += v*dt); true: history gate (x: older
+// snapshot, v: newer snapshot, dt unused; x <- v after the step).
 cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
                         const float* dt, const int32_t* step, int m, float eps, float* f,
-                        float* l1, uint8_t* mask, void* ws, cudaStream_t s);
+                        float* l1, uint8_t* mask, void* ws, cudaStream_t s, bool history);
 
 // Same kernel with its scratch in a static device array (no allocation, at
 // most gate_noalloc_max_chunks() chunks; calls must not overlap on the GPU).

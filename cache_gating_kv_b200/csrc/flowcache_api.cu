@@ -127,8 +127,33 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
   FC_CHECK_PTR(recompute);
   FC_CHECK_PTR(ws);
   return launched(fc::launch_gate(x, v, n_chunks, n_per_chunk, dt, step, m, eps, f, l1_rel,
-                                  recompute, ws, static_cast<cudaStream_t>(stream)),
+                                  recompute, ws, static_cast<cudaStream_t>(stream), false),
                   "fc_chunk_l1_gate");
+}
+
+fc_status fc_history_l1_gate(float* h_old, const float* h_new, int n_segments,
+                             int64_t n_per_segment, const int32_t* step, int32_t m, float delta,
+                             float* f, float* d_rel, uint8_t* refresh, void* ws, size_t ws_bytes,
+                             void* stream) {
+  fc::g_launches = 0;
+  if (n_segments < 1 || n_segments > 65535)
+    return fail(FC_ERR_INVALID_ARG, "n_segments must be in [1, 65535] (got %d)", n_segments);
+  if (n_per_segment < 0) return fail(FC_ERR_INVALID_ARG, "n_per_segment must be >= 0");
+  if (m < 0) return fail(FC_ERR_INVALID_ARG, "m must be >= 0");
+  if (ws == nullptr || ws_bytes < fc::gate_ws_bytes(n_segments))
+    return fail(FC_ERR_WORKSPACE, "gate workspace needs %zu bytes", fc::gate_ws_bytes(n_segments));
+  if (n_per_segment > 0) {
+    FC_CHECK_PTR(h_old);
+    FC_CHECK_PTR(h_new);
+  }
+  FC_CHECK_PTR(step);
+  FC_CHECK_PTR(f);
+  FC_CHECK_PTR(d_rel);
+  FC_CHECK_PTR(refresh);
+  FC_CHECK_PTR(ws);
+  return launched(fc::launch_gate(h_old, h_new, n_segments, n_per_segment, nullptr, step, m, delta,
+                                  f, d_rel, refresh, ws, static_cast<cudaStream_t>(stream), true),
+                  "fc_history_l1_gate");
 }
 
 fc_status fc_chunk_l1_gate_noalloc(float* x, const float* v, int n_chunks, int64_t n_per_chunk,

@@ -27,6 +27,10 @@ constexpr int kGateThreads = 256;
 constexpr int kGateUnroll = 4;
 constexpr int kGateMaxBlocksPerChunk = 1024;
 
+// kHist = false: the FlowCache gate (recompute resets f to 0).
+// kHist = true: the history-guided gate of the ARCache notes (关键设计 1,
+// HGC): a refresh step opens the next window, so f restarts at its own Delta.
+template <bool kHist>
 __device__ __forceinline__ void gate_finalize(int c, int st, int m, float eps, double num,
                                               double den, float* f, float* l1, uint8_t* mask) {
   float r;
@@ -35,14 +39,15 @@ __device__ __forceinline__ void gate_finalize(int c, int st, int m, float eps, d
   else
     r = (num > 0.0) ? __int_as_float(0x7f800000) : 0.0f;
   l1[c] = r;
+  const float reset = kHist ? r : 0.0f;
   if (st < m) {  // forced recompute during the first m steps of the chunk
     mask[c] = 1;
-    f[c] = 0.0f;
+    f[c] = reset;
   } else {
     const float acc = __fadd_rn(f[c], r);
     if (acc > eps) {  // recompute and reset
       mask[c] = 1;
-      f[c] = 0.0f;
+      f[c] = reset;
     } else {  // reuse, accumulate
       mask[c] = 0;
       f[c] = acc;
@@ -50,13 +55,18 @@ __device__ __forceinline__ void gate_finalize(int c, int st, int m, float eps, d
   }
 }
 
+// FlowCache: p = v*dt (rounded once), X <- X + p (rounded once).
+// History gate: p = h_t - h_{t+1} (rounded once), h_{t+1} <- h_t.
+// Both sum |p| and |X before the step| in float64.
+template <bool kHist>
 __device__ __forceinline__ void gate_elem(float& x, float vv, float h, double& num, double& den) {
-  const float p = __fmul_rn(vv, h);  // v*dt, rounded once
+  const float p = kHist ? __fsub_rn(vv, x) : __fmul_rn(vv, h);
   num += (double)fabsf(p);
   den += (double)fabsf(x);
-  x = __fadd_rn(x, p);  // X_{t-1} = X_t + v*dt, rounded once
+  x = kHist ? vv : __fadd_rn(x, p);
 }
 
+template <bool kHist>
 __global__ void __launch_bounds__(kGateThreads)
     gate_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t N,
                 const float* __restrict__ dt, const int32_t* __restrict__ step, int m, float eps,
@@ -73,7 +83,7 @@ __global__ void __launch_bounds__(kGateThreads)
     }
     return;
   }
-  const float h = dt[c];
+  const float h = kHist ? 0.0f : dt[c];
   const int64_t off = (int64_t)c * N;
   float* xc = x + off;
   const float* vc = v + off;
@@ -106,10 +116,10 @@ __global__ void __launch_bounds__(kGateThreads)
     for (int u = 0; u < kGateUnroll; ++u) {
       const int64_t i = base + (int64_t)u * kGateThreads;
       if (i < hi) {
-        gate_elem(xa[u].x, va[u].x, h, num, den);
-        gate_elem(xa[u].y, va[u].y, h, num, den);
-        gate_elem(xa[u].z, va[u].z, h, num, den);
-        gate_elem(xa[u].w, va[u].w, h, num, den);
+        gate_elem<kHist>(xa[u].x, va[u].x, h, num, den);
+        gate_elem<kHist>(xa[u].y, va[u].y, h, num, den);
+        gate_elem<kHist>(xa[u].z, va[u].z, h, num, den);
+        gate_elem<kHist>(xa[u].w, va[u].w, h, num, den);
         __stcs(x4 + i, xa[u]);
       }
     }
@@ -123,7 +133,7 @@ __global__ void __launch_bounds__(kGateThreads)
       e = tail0 + (tid - 4);
     if (e >= 0) {
       float xv = xc[e];
-      gate_elem(xv, vc[e], h, num, den);
+      gate_elem<kHist>(xv, vc[e], h, num, den);
       xc[e] = xv;
     }
   }
@@ -166,7 +176,7 @@ __global__ void __launch_bounds__(kGateThreads)
     a = warp_sum(a);
     d = warp_sum(d);
     if (lane == 0) {
-      gate_finalize(c, st, m, eps, a, d, f, l1, mask);
+      gate_finalize<kHist>(c, st, m, eps, a, d, f, l1, mask);
       counters[c] = 0u;  // ready for the next call
     }
   }
@@ -188,6 +198,7 @@ struct GateStage {
   float v[kSegFloats];
 };
 
+template <bool kHist>
 __global__ void __launch_bounds__(kTmaThreads, 1)
     gate_tma_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t N,
                     const float* __restrict__ dt, const int32_t* __restrict__ step, int m,
@@ -210,7 +221,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     }
     return;
   }
-  const float h = dt[c];
+  const float h = kHist ? 0.0f : dt[c];
   // This block's slice of the chunk, in whole vectors.
   const int64_t nvec = N >> 2;
   const int64_t per = ceil_div(nvec, bpc);
@@ -252,10 +263,10 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     float4* gx = reinterpret_cast<float4*>(xs + off);
     for (int i = tid; i < cnt4; i += kTmaThreads) {
       float4 xa = sx[i];
-      gate_elem(xa.x, sv[i].x, h, num, den);
-      gate_elem(xa.y, sv[i].y, h, num, den);
-      gate_elem(xa.z, sv[i].z, h, num, den);
-      gate_elem(xa.w, sv[i].w, h, num, den);
+      gate_elem<kHist>(xa.x, sv[i].x, h, num, den);
+      gate_elem<kHist>(xa.y, sv[i].y, h, num, den);
+      gate_elem<kHist>(xa.z, sv[i].z, h, num, den);
+      gate_elem<kHist>(xa.w, sv[i].w, h, num, den);
       __stcs(gx + i, xa);
     }
     __syncthreads();  // stage sidx fully consumed
@@ -295,7 +306,7 @@ __global__ void __launch_bounds__(kTmaThreads, 1)
     a = warp_sum(a);
     d = warp_sum(d);
     if (lane == 0) {
-      gate_finalize(c, st, m, eps, a, d, f, l1, mask);
+      gate_finalize<kHist>(c, st, m, eps, a, d, f, l1, mask);
       counters[c] = 0u;
     }
   }
@@ -314,7 +325,7 @@ size_t gate_ws_bytes(int n_chunks) {
 
 cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t N, const float* dt,
                         const int32_t* step, int m, float eps, float* f, float* l1,
-                        uint8_t* mask, void* ws, cudaStream_t s) {
+                        uint8_t* mask, void* ws, cudaStream_t s, bool history) {
   unsigned* counters = static_cast<unsigned*>(ws);
   int* err = reinterpret_cast<int*>(counters + n_chunks);
   double2* partials =
@@ -327,10 +338,11 @@ cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t N, const
     if (bpc < 1) bpc = 1;
     if (bpc > kGateMaxBlocksPerChunk) bpc = kGateMaxBlocksPerChunk;
     const size_t smem = (size_t)kSegStages * sizeof(GateStage) + kSegStages * sizeof(uint64_t);
-    cudaError_t e = cudaFuncSetAttribute(gate_tma_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = history ? gate_tma_kernel<true> : gate_tma_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
-    gate_tma_kernel<<<dim3((unsigned)bpc, (unsigned)n_chunks), kTmaThreads, smem, s>>>(
+    kern<<<dim3((unsigned)bpc, (unsigned)n_chunks), kTmaThreads, smem, s>>>(
         x, v, N, dt, step, m, eps, f, l1, mask, counters, partials, (int)bpc, err);
     add_launches(1);
     return cudaGetLastError();
@@ -343,8 +355,9 @@ cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t N, const
   if (bpc < 1) bpc = 1;
   if (bpc > kGateMaxBlocksPerChunk) bpc = kGateMaxBlocksPerChunk;
   dim3 grid((unsigned)bpc, (unsigned)n_chunks);
-  gate_kernel<<<grid, kGateThreads, 0, s>>>(x, v, N, dt, step, m, eps, f, l1, mask, counters,
-                                            partials, (int)bpc);
+  auto kern = history ? gate_kernel<true> : gate_kernel<false>;
+  kern<<<grid, kGateThreads, 0, s>>>(x, v, N, dt, step, m, eps, f, l1, mask, counters, partials,
+                                     (int)bpc);
   add_launches(1);
   return cudaGetLastError();
 }
@@ -400,7 +413,7 @@ cudaError_t launch_gate_noalloc(float* x, const float* v, int n_chunks, int64_t 
   e = cudaMemsetAsync(ws, 0, (size_t)(n_chunks + 1) * sizeof(unsigned), s);
   if (e != cudaSuccess) return e;
   add_launches(1);
-  return launch_gate(x, v, n_chunks, N, dt, step, m, eps, f, l1, mask, ws, s);
+  return launch_gate(x, v, n_chunks, N, dt, step, m, eps, f, l1, mask, ws, s, false);
 }
 
 }  // namespace fc

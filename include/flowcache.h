@@ -116,6 +116,35 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
                            size_t ws_bytes, void* stream);
 
 /*
+ * History-guided variant of the gate, for the neighbouring method of the notes
+ * "Accelerating Autoregressive Video Diffusion via History-Guided Cache and
+ * Residual Correction" (papernotes.org), 关键设计 1 (HGC).  Per segment:
+ *   Delta = ||h_t - h_{t+1}||_1 / ||h_{t+1}||_1  (denominator: the older step),
+ * and the cache refreshes at the step where the deviations summed since the
+ * last refresh step t_ref (inclusive) first exceed delta:
+ *   sum_{i=t+1}^{t_ref} Delta <= delta < sum_{i=t}^{t_ref} Delta.
+ * The refresh step becomes t_ref, so f restarts at that step's own Delta
+ * (where fc_chunk_l1_gate resets to 0).  The first m steps of a segment
+ * refresh unconditionally.  Same kernels, reductions and precision as
+ * fc_chunk_l1_gate: h_t - h_{t+1} is rounded once in float32, both norms are
+ * summed in float64, the recurrence runs in float32.
+ *
+ *   h_old     [n][N] float32, in/out: h_{t+1} in, h_t out (for active segments)
+ *   h_new     [n][N] float32, h_t
+ *   step      [n] int32, steps since the segment started; < 0: inactive, untouched
+ *   m, delta  forced refresh steps, threshold
+ *   f         [n] float32, in/out window sum
+ *   d_rel     [n] float32, out: Delta
+ *   refresh   [n] uint8, out: 1 = refresh (recompute) at this step
+ *   ws        fc_gate_workspace_size(n, N) bytes, same contract as the gate's
+ * Errors as for fc_chunk_l1_gate.
+ */
+fc_status fc_history_l1_gate(float* h_old, const float* h_new, int n_segments,
+                             int64_t n_per_segment, const int32_t* step, int32_t m, float delta,
+                             float* f, float* d_rel, uint8_t* refresh, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/*
  * Allocation-free variant of fc_chunk_l1_gate.  The paper has no counterpart:
  * this entry point exists for callers that cannot allocate device memory when
  * they run the gate -- for example a host runtime that hands its plugins only

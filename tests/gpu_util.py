@@ -97,3 +97,19 @@ def assert_selection_matches(idx_gpu, score_ref, B, tol):
         assert gs.issuperset(ref_keep.tolist()), f"head {h}: a clear keeper was dropped"
         assert not gs.intersection(ref_drop.tolist()), f"head {h}: a clear loser was kept"
         assert len(gs) == B
+
+
+def history_gate_gpu(h_old, h_new, step, m, delta, f, ws=None):
+    """One history-gate step on the GPU; returns numpy (h_next, f_next, d, refresh)."""
+    ho = torch.from_numpy(np.ascontiguousarray(h_old, np.float32)).to(DEV)
+    hn = torch.from_numpy(np.ascontiguousarray(h_new, np.float32)).to(DEV)
+    n = ho.shape[0]
+    sd = torch.from_numpy(np.asarray(step, np.int32)).to(DEV)
+    fd = torch.from_numpy(np.asarray(f, np.float32).copy()).to(DEV)
+    d = torch.full((n,), -1.0, device=DEV)
+    r = torch.full((n,), 7, dtype=torch.uint8, device=DEV)
+    if ws is None:
+        ws = fc.workspace(fc.fc_gate_workspace_size(n, ho.shape[1]))
+    fc.fc_history_l1_gate(ho, hn, sd, m, delta, fd, d, r, ws)
+    torch.cuda.synchronize()
+    return ho.cpu().numpy(), fd.cpu().numpy(), d.cpu().numpy(), r.cpu().numpy()

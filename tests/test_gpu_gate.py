@@ -130,3 +130,45 @@ def test_gate_deterministic_and_counters_reset():
     for u, w in zip(a, b):
         np.testing.assert_array_equal(u, w)
     assert int(ws[: 4 * (cfg.n_chunks + 1)].sum()) == 0  # counters back at zero, no error
+
+
+# ---------------------------------------------------------------------------
+# history-guided gate (fc_history_l1_gate)
+# ---------------------------------------------------------------------------
+def test_history_gate_hand_trace_on_gpu(golden_dir):
+    from tests.gpu_util import history_gate_gpu
+    g = json.load(open(os.path.join(golden_dir, "history_gate_trace.json")))
+    N = g["N"]
+    f = np.zeros(1, np.float32)
+    for t in range(g["steps"]):
+        h_old = np.full((1, N), g["h_old"], np.float32)
+        h_new = np.full((1, N), g["h_new"], np.float32)
+        hn, f, d, mask = history_gate_gpu(h_old, h_new, [t], g["m"], g["delta"], f)
+        assert d[0] == np.float32(g["d"]) and mask[0] == g["mask"][t] and f[0] == np.float32(g["f"][t])
+        assert np.all(hn == np.float32(g["h_new"]))
+
+
+@pytest.mark.parametrize("n,N", [(4, 777600), (3, 1001), (5, 4096), (16, 24 * 45 * 45 * 16 // 8)])
+def test_history_gate_trajectory_parity(n, N):
+    """History snapshots drifting over 12 steps; GPU and oracle side by side."""
+    from tests.gpu_util import history_gate_gpu
+    rng = np.random.default_rng(n * 7 + N)
+    h_r = h_g = rng.standard_normal((n, N)).astype(np.float32)
+    f_r = f_g = np.zeros(n, np.float32)
+    delta = 0.05
+    ws = fc.workspace(fc.fc_gate_workspace_size(n, N))
+    for t in range(12):
+        h_new = (h_r + rng.standard_normal((n, N)).astype(np.float32) *
+                 np.float32(0.004 * (1 + t % 3))).astype(np.float32)
+        step = np.where(np.arange(n) == n - 1, -1 if t < 3 else t - 3, t).astype(np.int32)
+        ref = O.history_gate_step(h_r, h_new, step, 1, delta, f_r)
+        got = history_gate_gpu(h_g, h_new, step, 1, delta, f_g, ws=ws)
+        np.testing.assert_array_equal(got[0].view(np.uint32), ref[0].view(np.uint32))
+        np.testing.assert_allclose(got[2], ref[2], rtol=1e-6)
+        for c in range(n):
+            margin = abs(float(np.float32(f_r[c] + ref[2][c])) - delta) if step[c] >= 1 else 1.0
+            if margin < MARGIN:
+                continue
+            assert got[3][c] == ref[3][c] and got[1][c] == pytest.approx(ref[1][c], rel=1e-6)
+        h_r, f_r = ref[0], ref[1]
+        h_g, f_g = got[0], got[1]
