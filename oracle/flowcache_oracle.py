@@ -47,6 +47,8 @@ import numpy as np
 __all__ = [
     "gate_step",
     "history_gate_step",
+    "gather_recompute",
+    "scatter_velocity",
     "importance",
     "row_lse",
     "importance_at",
@@ -168,6 +170,34 @@ def history_gate_step(h_old, h_new, step, m, delta, f):
             mask[c] = 0
             f_next[c] = acc
     return h_next, f_next, d, mask
+
+
+def gather_recompute(x, mask):
+    """The chunks the gate marked for recompute (key design 2 and the
+    flowchart: recompute chunks run the model forward, reuse chunks take their
+    cached activations), gathered in chunk order into a dense batch.
+
+    x [n_c, N], mask [n_c] uint8.  Returns (ids int32 [n_c] -- the recompute
+    chunk indices ascending, then -1 --, count, dense [n_c, N]); only the first
+    count rows of dense are part of the result."""
+    x = np.asarray(x)
+    n_c = x.shape[0]
+    ids = np.full(n_c, -1, dtype=np.int32)
+    sel = [c for c in range(n_c) if mask[c] != 0]
+    ids[:len(sel)] = sel
+    dense = np.zeros_like(x)
+    for i, c in enumerate(sel):
+        dense[i] = x[c]
+    return ids, len(sel), dense
+
+
+def scatter_velocity(v_cache, v_dense, ids, count):
+    """Fresh velocities of the recomputed chunks back into the per-chunk cache:
+    v_cache[ids[i]] = v_dense[i] for i < count; reused chunks keep theirs."""
+    out = np.array(v_cache, copy=True)
+    for i in range(count):
+        out[ids[i]] = v_dense[i]
+    return out
 
 
 # ---------------------------------------------------------------------------

@@ -431,3 +431,23 @@ def test_history_gate_matches_cumulative_rule_brute_force():
             else:
                 exp.append(0)
         assert [m for m, _ in got] == exp
+
+
+# ---------------------------------------------------------------------------
+# Gate-mask consumer: gather / scatter around the model forward
+# ---------------------------------------------------------------------------
+def test_gather_scatter_round_trip():
+    rng = np.random.default_rng(21)
+    x = rng.standard_normal((6, 10)).astype(np.float32)
+    mask = np.array([0, 1, 1, 0, 0, 1], np.uint8)
+    ids, count, dense = O.gather_recompute(x, mask)
+    assert count == 3 and list(ids) == [1, 2, 5, -1, -1, -1]
+    np.testing.assert_array_equal(dense[:3], x[[1, 2, 5]])
+    assert np.all(dense[3:] == 0)
+    v_cache = rng.standard_normal((6, 10)).astype(np.float32)
+    fresh = rng.standard_normal((6, 10)).astype(np.float32)
+    out = O.scatter_velocity(v_cache, fresh, ids, count)
+    np.testing.assert_array_equal(out[[1, 2, 5]], fresh[:3])
+    np.testing.assert_array_equal(out[[0, 3, 4]], v_cache[[0, 3, 4]])
+    ids0, c0, d0 = O.gather_recompute(x, np.zeros(6, np.uint8))
+    assert c0 == 0 and np.all(ids0 == -1) and np.all(d0 == 0)
