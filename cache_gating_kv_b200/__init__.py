@@ -26,6 +26,8 @@ __all__ = [
     "fc_chunk_l1_gate",
     "fc_chunk_l1_gate_noalloc",
     "fc_history_l1_gate",
+    "fc_gather_recompute",
+    "fc_scatter_velocity",
     "fc_kv_importance",
     "fc_kv_redundancy",
     "fc_kv_score_topb",
@@ -67,6 +69,8 @@ def _declare(lib):
                                              c_f, c_p, c_p, c_p, c_p]),
         "fc_history_l1_gate": (c_int, [c_p, c_p, c_int, c_i64, c_p, ctypes.c_int32, c_f, c_p, c_p,
                                        c_p, c_p, c_sz, c_p]),
+        "fc_gather_recompute": (c_int, [c_p, c_p, c_int, c_i64, c_p, c_p, c_p, c_p]),
+        "fc_scatter_velocity": (c_int, [c_p, c_p, c_p, c_int, c_i64, c_p, c_p]),
         "fc_importance_workspace_size": (c_sz, [c_int, c_int, c_int, c_int, c_int]),
         "fc_kv_importance": (c_int, [c_p, c_p, c_int, c_int, c_int, c_int, c_int, c_f, c_p, c_p,
                                      c_sz, c_p]),
@@ -194,6 +198,23 @@ def fc_chunk_l1_gate_noalloc(x, v, dt, step, m, eps, f, l1_rel, recompute, strea
                                              float(eps), _p(f), _p(l1_rel), _p(recompute),
                                              _s(stream))
     _check("fc_chunk_l1_gate_noalloc", st)
+
+
+def fc_gather_recompute(x, recompute, dense, ids, count, stream=None):
+    """Gather the recompute chunks' rows of x [n_c, N] into dense [n_c, N];
+    ids [n_c] int32 and count [1] int32 are written on the device."""
+    n_c, N = x.shape
+    st = library().fc_gather_recompute(_p(x), _p(recompute), n_c, N, _p(dense), _p(ids),
+                                        _p(count), _s(stream))
+    _check("fc_gather_recompute", st)
+
+
+def fc_scatter_velocity(v_dense, ids, count, v_cache, stream=None):
+    """v_cache[ids[i]] = v_dense[i] for i < count (device-side count)."""
+    n_c, N = v_cache.shape
+    st = library().fc_scatter_velocity(_p(v_dense), _p(ids), _p(count), n_c, N, _p(v_cache),
+                                        _s(stream))
+    _check("fc_scatter_velocity", st)
 
 
 def fc_kv_importance(q, k, imp, ws, scale=0.0, stream=None):

@@ -23,6 +23,12 @@ cudaError_t launch_gate_noalloc(float* x, const float* v, int n_chunks, int64_t 
                                 const float* dt, const int32_t* step, int m, float eps, float* f,
                                 float* l1, uint8_t* mask, cudaStream_t s);
 
+// ---- consumer of the recompute mask ------------------------------------------
+cudaError_t launch_gather_recompute(const float* x, const uint8_t* mask, int n_c, int64_t N,
+                                    float* dense, int32_t* ids, int32_t* count, cudaStream_t s);
+cudaError_t launch_scatter_velocity(const float* v_dense, const int32_t* ids, const int32_t* count,
+                                    int n_c, int64_t N, float* v_cache, cudaStream_t s);
+
 // ---- importance --------------------------------------------------------------
 size_t importance_ws_bytes(int H, int Lq);
 // bf16 tensor-core path (tcgen05 + TMEM + TMA)

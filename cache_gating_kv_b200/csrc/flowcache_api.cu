@@ -182,6 +182,45 @@ fc_status fc_chunk_l1_gate_noalloc(float* x, const float* v, int n_chunks, int64
                   "fc_chunk_l1_gate_noalloc");
 }
 
+fc_status fc_gather_recompute(const float* x, const uint8_t* recompute, int n_chunks,
+                              int64_t n_per_chunk, float* dense, int32_t* ids, int32_t* count,
+                              void* stream) {
+  fc::g_launches = 0;
+  if (n_chunks < 1 || n_chunks > 65535)
+    return fail(FC_ERR_INVALID_ARG, "n_chunks must be in [1, 65535] (got %d)", n_chunks);
+  if (n_per_chunk < 0) return fail(FC_ERR_INVALID_ARG, "n_per_chunk must be >= 0");
+  if (n_per_chunk > 0) {
+    FC_CHECK_PTR(x);
+    FC_CHECK_PTR(dense);
+  }
+  FC_CHECK_PTR(recompute);
+  FC_CHECK_PTR(ids);
+  FC_CHECK_PTR(count);
+  return launched(fc::launch_gather_recompute(x, recompute, n_chunks, n_per_chunk, dense, ids,
+                                              count, static_cast<cudaStream_t>(stream)),
+                  "fc_gather_recompute");
+}
+
+fc_status fc_scatter_velocity(const float* v_dense, const int32_t* ids, const int32_t* count,
+                              int n_chunks, int64_t n_per_chunk, float* v_cache, void* stream) {
+  fc::g_launches = 0;
+  if (n_chunks < 1 || n_chunks > 65535)
+    return fail(FC_ERR_INVALID_ARG, "n_chunks must be in [1, 65535] (got %d)", n_chunks);
+  if (n_per_chunk < 0) return fail(FC_ERR_INVALID_ARG, "n_per_chunk must be >= 0");
+  if (n_per_chunk > 0) {
+    FC_CHECK_PTR(v_dense);
+    FC_CHECK_PTR(v_cache);
+  }
+  FC_CHECK_PTR(ids);
+  FC_CHECK_PTR(count);
+  const size_t bytes = (size_t)n_chunks * n_per_chunk * sizeof(float);
+  if (n_per_chunk > 0 && ranges_overlap(v_dense, bytes, v_cache, bytes))
+    return fail(FC_ERR_INVALID_ARG, "v_dense and v_cache overlap");
+  return launched(fc::launch_scatter_velocity(v_dense, ids, count, n_chunks, n_per_chunk, v_cache,
+                                              static_cast<cudaStream_t>(stream)),
+                  "fc_scatter_velocity");
+}
+
 size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d) {
   (void)dtype;
   (void)Lk;

@@ -172,6 +172,36 @@ fc_status fc_chunk_l1_gate_noalloc(float* x, const float* v, int n_chunks, int64
                                    const float* dt, const int32_t* step, int32_t m, float eps,
                                    float* f, float* l1_rel, uint8_t* recompute, void* stream);
 
+/*
+ * Consumer of the recompute mask (the flowchart of 整体框架 and key design 2:
+ * chunks marked for recompute run the model forward, the others reuse their
+ * cached activations).  Gathers, in chunk order, the latents of the chunks
+ * with recompute[c] != 0 into the first rows of a dense batch.
+ *
+ *   x          [n_chunks][n_per_chunk] float32
+ *   recompute  [n_chunks] uint8 (the gate's output)
+ *   dense      [n_chunks][n_per_chunk] float32 out: rows 0..count-1 are the
+ *              recompute chunks' latents; rows >= count are not written
+ *   ids        [n_chunks] int32 out: ids[i] = chunk of dense row i, -1 past count
+ *   count      [1] int32 out (device): number of recompute chunks
+ * Everything stays on the device (no host synchronisation).  Bitwise copy.
+ * Errors: bad sizes or pointers -> FC_ERR_INVALID_ARG.
+ */
+fc_status fc_gather_recompute(const float* x, const uint8_t* recompute, int n_chunks,
+                              int64_t n_per_chunk, float* dense, int32_t* ids, int32_t* count,
+                              void* stream);
+
+/*
+ * The other half: after the forward of the dense batch, v_cache[ids[i]] =
+ * v_dense[i] for i < *count; the reused chunks keep their cached velocity.
+ *
+ *   v_dense  [n_chunks][n_per_chunk] float32, fresh velocities of the batch
+ *   ids, count  as written by fc_gather_recompute
+ *   v_cache  [n_chunks][n_per_chunk] float32 in/out; must not overlap v_dense
+ */
+fc_status fc_scatter_velocity(const float* v_dense, const int32_t* ids, const int32_t* count,
+                              int n_chunks, int64_t n_per_chunk, float* v_cache, void* stream);
+
 /* ------------------------------------------------------------------------ */
 /* Joint importance-redundancy KV compression (key design 3)                */
 /* ------------------------------------------------------------------------ */

@@ -129,3 +129,17 @@ def test_selftest_entries_validate_on_the_host():
     lib.fc_selftest_exp2.restype = C.c_int
     lib.fc_selftest_exp2.argtypes = [C.c_void_p] * 3 + [C.c_int, C.c_void_p]
     assert lib.fc_selftest_exp2(None, None, None, 3, None) == 1  # odd n
+
+
+def test_mask_consumer_validates_on_the_host():
+    lib = fc.library()
+    # n_chunks out of range
+    assert lib.fc_gather_recompute(NULL, NULL, 0, 8, NULL, NULL, NULL, NULL) == 1
+    assert lib.fc_gather_recompute(NULL, NULL, 70000, 8, NULL, NULL, NULL, NULL) == 1
+    assert lib.fc_scatter_velocity(NULL, NULL, NULL, 0, 8, NULL, NULL) == 1
+    # negative size, NULL buffers
+    assert lib.fc_gather_recompute(NULL, NULL, 4, -1, NULL, NULL, NULL, NULL) == 1
+    assert lib.fc_gather_recompute(NULL, NULL, 4, 8, NULL, NULL, NULL, NULL) == 1
+    assert lib.fc_last_error() == b"x is NULL"
+    assert lib.fc_scatter_velocity(NULL, NULL, NULL, 4, 8, NULL, NULL) == 1
+    assert lib.fc_last_error() == b"v_dense is NULL"
