@@ -49,6 +49,8 @@ __all__ = [
     "history_gate_step",
     "gather_recompute",
     "scatter_velocity",
+    "cache_commit",
+    "cache_stream",
     "importance",
     "row_lse",
     "importance_at",
@@ -376,3 +378,59 @@ def compact(k, v, idx):
                 k_out[h, r] = k[h, j]
                 v_out[h, r] = v[h, j]
     return k_out, v_out
+
+
+# ---------------------------------------------------------------------------
+# Cache buffer management around compression (key design 3 and the flowchart:
+# a finished chunk enters the KV cache; when the reserved cache is full it is
+# merged into the candidates and each head keeps its top-B tokens)
+# ---------------------------------------------------------------------------
+
+def cache_commit(k_buf, v_buf, n_clean, C, B_budget, q, lam, window, scale=None):
+    """One finished chunk enters the fixed buffer ``B_total = B_budget + C``.
+
+    k_buf, v_buf [H, B_budget + C, d]: rows [0, n_clean) hold the compressed
+    clean tokens, rows [n_clean, n_clean + C) the chunk that has just finished
+    denoising.  q [H, L_q, d] are the queries of the chunk now denoising.
+
+    If the n_clean + C candidates fit in B_budget they are kept as they are:
+    returns (k_buf, v_buf, n_clean + C, None).  Otherwise the candidates are
+    scored (importance of q over them, redundancy, joint score) and every head
+    keeps its top-B_budget; returns (k_next, v_next, B_budget, idx) with the
+    kept rows in rows [0, B_budget) of new buffers of the same shape, the rest
+    zero, and idx [H, B_budget] the kept candidate rows."""
+    H, cap, d = k_buf.shape
+    assert cap == B_budget + C and 0 <= n_clean <= B_budget
+    L = n_clean + C
+    if L <= B_budget:
+        return k_buf, v_buf, L, None
+    kc, vc = k_buf[:, :L], v_buf[:, :L]
+    imp = importance(q, kc, scale)
+    red = redundancy(kc)
+    _, idx = score_topb(imp, red, lam, window, B_budget)
+    ko, vo = compact(kc, vc, idx)
+    k_next = np.zeros_like(k_buf)
+    v_next = np.zeros_like(v_buf)
+    k_next[:, :B_budget] = ko
+    v_next[:, :B_budget] = vo
+    return k_next, v_next, B_budget, idx
+
+
+def cache_stream(chunks_k, chunks_v, queries, B_budget, lam, window, scale=None):
+    """Chunks finish one after another: chunk i's K/V [H, C, d] go into the
+    active rows, then ``cache_commit`` with queries[i].  Returns the final
+    (k_buf, v_buf, n_clean) and the clean length after each chunk."""
+    H, C, d = chunks_k[0].shape
+    k_buf = np.zeros((H, B_budget + C, d), dtype=chunks_k[0].dtype)
+    v_buf = np.zeros_like(k_buf)
+    n = 0
+    lengths = []
+    for kc, vc, q in zip(chunks_k, chunks_v, queries):
+        k_buf = k_buf.copy()
+        v_buf = v_buf.copy()
+        k_buf[:, n:n + C] = kc
+        v_buf[:, n:n + C] = vc
+        k_buf, v_buf, n, _ = cache_commit(k_buf, v_buf, n, C, B_budget, q, lam, window, scale)
+        lengths.append(n)
+    return k_buf, v_buf, n, lengths
+

@@ -451,3 +451,69 @@ def test_gather_scatter_round_trip():
     np.testing.assert_array_equal(out[[0, 3, 4]], v_cache[[0, 3, 4]])
     ids0, c0, d0 = O.gather_recompute(x, np.zeros(6, np.uint8))
     assert c0 == 0 and np.all(ids0 == -1) and np.all(d0 == 0)
+
+
+# ---- cache buffer management -------------------------------------------------
+
+def _stream_inputs(H, C, d, n_chunks, Lq, seed, same_query=False):
+    rng = np.random.default_rng(seed)
+    ks = [rng.standard_normal((H, C, d)) for _ in range(n_chunks)]
+    vs = [rng.standard_normal((H, C, d)) for _ in range(n_chunks)]
+    if same_query:
+        q0 = rng.standard_normal((H, 1, d))
+        qs = [np.repeat(q0, Lq, axis=1) for _ in range(n_chunks)]
+    else:
+        qs = [rng.standard_normal((H, Lq, d)) for _ in range(n_chunks)]
+    return ks, vs, qs
+
+
+def test_cache_fills_then_holds_the_budget():
+    """The clean length grows by one chunk while it fits, then stays at
+    B_budget; before the first compression the buffer is the chunks in order."""
+    H, C, d, B = 2, 4, 8, 12
+    ks, vs, qs = _stream_inputs(H, C, d, 7, 3, seed=0)
+    _, _, n, lengths = O.cache_stream(ks, vs, qs, B, 0.5, 3)
+    assert lengths == [4, 8, 12, 12, 12, 12, 12] and n == 12
+    kb, vb, n, _ = O.cache_stream(ks[:3], vs[:3], qs[:3], B, 0.5, 3)
+    np.testing.assert_array_equal(kb[:, :12], np.concatenate(ks[:3], axis=1))
+    np.testing.assert_array_equal(vb[:, :12], np.concatenate(vs[:3], axis=1))
+
+
+def test_cache_importance_only_keeps_global_top_b_by_dot_product():
+    """lambda = 1, no pooling and one query repeated: the softmax is monotone
+    in q.k, so each compression keeps the B largest q.k among its candidates,
+    and over the stream the clean set is the B largest q.k of all tokens seen,
+    in the order they arrived (brute force over the concatenated tokens)."""
+    H, C, d, B, n_chunks = 3, 4, 8, 8, 6
+    ks, vs, qs = _stream_inputs(H, C, d, n_chunks, 5, seed=1, same_query=True)
+    kb, vb, n, _ = O.cache_stream(ks, vs, qs, B, 1.0, 1)
+    allk = np.concatenate(ks, axis=1)
+    allv = np.concatenate(vs, axis=1)
+    for h in range(H):
+        dots = allk[h] @ qs[0][h, 0]
+        keep = np.sort(np.argsort(-dots)[:B])
+        np.testing.assert_array_equal(kb[h, :B], allk[h, keep])
+        np.testing.assert_array_equal(vb[h, :B], allv[h, keep])
+
+
+def test_cache_redundancy_only_drops_the_repeated_key():
+    """lambda = 0: the score is minus the redundancy.  Candidates
+    [e1, e1, e2, e1, e3, e4]: each copy of e1 has cosine row sum 2, the others
+    0, so the three kept are e2, e3, e4 (candidate rows 2, 4, 5)."""
+    e = np.eye(4)
+    k1 = np.stack([e[0], e[0], e[1]])[None]
+    k2 = np.stack([e[0], e[2], e[3]])[None]
+    v1, v2 = k1 * 10, k2 * 10
+    q = np.ones((1, 2, 4))
+    kb = np.zeros((1, 6, 4))
+    vb = np.zeros((1, 6, 4))
+    kb[:, :3], vb[:, :3] = k1, v1
+    kb, vb, n, idx = O.cache_commit(kb, vb, 0, 3, 3, q, 0.0, 1)
+    assert n == 3 and idx is None
+    kb[:, 3:], vb[:, 3:] = k2, v2
+    kn, vn, n, idx = O.cache_commit(kb, vb, 3, 3, 3, q, 0.0, 1)
+    assert n == 3
+    np.testing.assert_array_equal(idx, [[2, 4, 5]])
+    np.testing.assert_array_equal(kn[0, :3], np.stack([e[1], e[2], e[3]]))
+    np.testing.assert_array_equal(vn[0, :3], 10 * np.stack([e[1], e[2], e[3]]))
+    assert not kn[:, 3:].any()
