@@ -28,6 +28,8 @@ __all__ = [
     "fc_history_l1_gate",
     "fc_gather_recompute",
     "fc_scatter_velocity",
+    "fc_kv_cache_workspace_size",
+    "fc_kv_cache_commit",
     "fc_kv_importance",
     "fc_kv_redundancy",
     "fc_kv_score_topb",
@@ -81,6 +83,10 @@ def _declare(lib):
                                      c_sz, c_p]),
         "fc_kv_compact": (c_int, [c_p, c_p, c_int, c_int, c_int, c_int, c_p, c_int, c_p, c_p,
                                   c_p]),
+        "fc_kv_cache_workspace_size": (c_sz, [c_int, c_int, c_int, c_int, c_int, c_int]),
+        "fc_kv_cache_commit": (c_int, [c_p, c_p, c_p, c_p, c_p, c_int, c_int, c_int, c_int, c_int,
+                                       c_int, c_int, c_f, c_int, c_f, c_p, c_p, c_sz,
+                                       ctypes.POINTER(c_int), ctypes.POINTER(c_int), c_p]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -158,6 +164,10 @@ def fc_redundancy_workspace_size(dtype, H, Lk, d):
 
 def fc_score_topb_workspace_size(H, Lk, B):
     return library().fc_score_topb_workspace_size(H, Lk, B)
+
+
+def fc_kv_cache_workspace_size(dtype, H, Lq, B_budget, C, d):
+    return library().fc_kv_cache_workspace_size(dtype, H, Lq, B_budget, C, d)
 
 
 def workspace(nbytes, device=None):
@@ -242,6 +252,22 @@ def fc_kv_score_topb(imp, red, pool_window, lam, B, idx, ws, score=None, stream=
     st = library().fc_kv_score_topb(_p(imp), _p(red), H, Lk, int(pool_window), float(lam), int(B),
                                      _p(score), _p(idx), _p(ws), ws.numel(), _s(stream))
     _check("fc_kv_score_topb", st)
+
+
+def fc_kv_cache_commit(q, k_buf, v_buf, k_next, v_next, n_clean, C, ws, pool_window, lam,
+                       scale=0.0, idx=None, stream=None):
+    """One finished chunk enters the cache buffer [H, B_budget + C, d]; returns
+    (n_next, compressed).  When compressed, the kept rows are in rows
+    [0, B_budget) of k_next / v_next and the caller swaps the buffers."""
+    H, cap, d = k_buf.shape
+    Lq = q.shape[1]
+    n_next, comp = ctypes.c_int(-1), ctypes.c_int(-1)
+    st = library().fc_kv_cache_commit(
+        _p(q), _p(k_buf), _p(v_buf), _p(k_next), _p(v_next), _dtype_code(k_buf), H, Lq, d,
+        cap - C, C, n_clean, float(scale), int(pool_window), float(lam), _p(idx), _p(ws),
+        0 if ws is None else ws.numel() * ws.element_size(), ctypes.byref(n_next), ctypes.byref(comp), _s(stream))
+    _check("fc_kv_cache_commit", st)
+    return n_next.value, bool(comp.value)
 
 
 def fc_kv_compact(k, v, idx, k_out, v_out, stream=None):

@@ -58,6 +58,7 @@ cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk,
 
 // ---- compaction ------------------------------------------------------------------
 cudaError_t launch_compact(const void* k, const void* v, int elem_bytes, int H, int Lk, int d,
-                           const int32_t* idx, int B, void* k_out, void* v_out, cudaStream_t s);
+                           const int32_t* idx, int B, int ldo, void* k_out, void* v_out,
+                           cudaStream_t s);
 
 }  // namespace fc

@@ -90,6 +90,30 @@ fc_status check_kv_shape(fc_dtype dtype, int H, int L1, int L2, int d) {
   return FC_OK;
 }
 
+// Workspace of fc_kv_cache_commit: the importance stage's own workspace first
+// (so bytes 0..3 are its error word, as for fc_kv_importance), then Imp, Red
+// and the selection, then the redundancy and score/top-B workspaces.
+struct CacheWs {
+  size_t imp, red, idx, red_ws, score_ws, total;
+};
+
+CacheWs cache_ws(int H, int Lq, int B_budget, int C, int d) {
+  const size_t cap = (size_t)B_budget + C;
+  CacheWs w;
+  size_t o = fc::align_up(fc::importance_ws_bytes(H, Lq), 256);
+  w.imp = o;
+  o = fc::align_up(o + (size_t)H * cap * sizeof(float), 256);
+  w.red = o;
+  o = fc::align_up(o + (size_t)H * cap * sizeof(float), 256);
+  w.idx = o;
+  o = fc::align_up(o + (size_t)H * B_budget * sizeof(int32_t), 256);
+  w.red_ws = o;
+  o = fc::align_up(o + fc::redundancy_ws_bytes(H, d), 256);
+  w.score_ws = o;
+  w.total = fc::align_up(o + fc::score_topb_ws_bytes(H, (int)cap), 256);
+  return w;
+}
+
 }  // namespace
 
 extern "C" {
@@ -317,9 +341,84 @@ fc_status fc_kv_compact(const void* k, const void* v, fc_dtype dtype, int H, int
       ranges_overlap(v_out, out_bytes, k, in_bytes) || ranges_overlap(v_out, out_bytes, v, in_bytes) ||
       ranges_overlap(k_out, out_bytes, v_out, out_bytes))
     return fail(FC_ERR_INVALID_ARG, "k_out / v_out overlap an input or each other");
-  return launched(fc::launch_compact(k, v, (int)elem_bytes(dtype), H, Lk, d, idx, B, k_out, v_out,
-                                     static_cast<cudaStream_t>(stream)),
+  return launched(fc::launch_compact(k, v, (int)elem_bytes(dtype), H, Lk, d, idx, B, B, k_out,
+                                     v_out, static_cast<cudaStream_t>(stream)),
                   "fc_kv_compact");
+}
+
+size_t fc_kv_cache_workspace_size(fc_dtype dtype, int H, int Lq, int B_budget, int C, int d) {
+  (void)dtype;
+  if (H < 1 || Lq < 1 || B_budget < 1 || C < 1 || (d != 64 && d != 128)) return 0;
+  return cache_ws(H, Lq, B_budget, C, d).total;
+}
+
+fc_status fc_kv_cache_commit(const void* q, const void* k_buf, const void* v_buf, void* k_next,
+                             void* v_next, fc_dtype dtype, int H, int Lq, int d, int B_budget,
+                             int C, int n_clean, float scale, int pool_window, float lambda,
+                             int32_t* idx, void* ws, size_t ws_bytes, int* n_next,
+                             int* compressed, void* stream) {
+  fc::g_launches = 0;
+  if (n_next == nullptr || compressed == nullptr)
+    return fail(FC_ERR_INVALID_ARG, "n_next and compressed must be host pointers");
+  if (C < 1 || B_budget < C)
+    return fail(FC_ERR_INVALID_ARG, "need 1 <= C <= B_budget (got C=%d, B_budget=%d)", C, B_budget);
+  if ((int64_t)B_budget + C > INT32_MAX / 2) return fail(FC_ERR_INVALID_ARG, "B_budget + C too large");
+  const int cap = B_budget + C;
+  fc_status st = check_kv_shape(dtype, H, Lq, cap, d);
+  if (st != FC_OK) return st;
+  if (B_budget % C != 0)
+    return fail(FC_ERR_UNSUPPORTED, "B_budget (%d) must be a multiple of C (%d)", B_budget, C);
+  if (n_clean < 0 || n_clean > B_budget || n_clean % C != 0)
+    return fail(FC_ERR_INVALID_ARG, "n_clean must be a multiple of C in [0, B_budget] (got %d)",
+                n_clean);
+  if (pool_window < 1 || pool_window % 2 == 0 || pool_window > 511)
+    return fail(FC_ERR_INVALID_ARG, "pool_window must be odd and in [1, 511] (got %d)",
+                pool_window);
+  if (n_clean + C <= B_budget) {  // the chunk fits: it stays where it is
+    *n_next = n_clean + C;
+    *compressed = 0;
+    return ok();
+  }
+  const CacheWs lay = cache_ws(H, Lq, B_budget, C, d);
+  if (ws == nullptr || ws_bytes < lay.total)
+    return fail(FC_ERR_WORKSPACE, "cache workspace needs %zu bytes", lay.total);
+  FC_CHECK_PTR(q);
+  FC_CHECK_PTR(k_buf);
+  FC_CHECK_PTR(v_buf);
+  FC_CHECK_PTR(k_next);
+  FC_CHECK_PTR(v_next);
+  FC_CHECK_PTR(ws);
+  if (idx != nullptr) FC_CHECK_PTR(idx);
+  const size_t buf_bytes = (size_t)H * cap * d * elem_bytes(dtype);
+  if (ranges_overlap(k_next, buf_bytes, k_buf, buf_bytes) ||
+      ranges_overlap(k_next, buf_bytes, v_buf, buf_bytes) ||
+      ranges_overlap(v_next, buf_bytes, k_buf, buf_bytes) ||
+      ranges_overlap(v_next, buf_bytes, v_buf, buf_bytes) ||
+      ranges_overlap(k_next, buf_bytes, v_next, buf_bytes))
+    return fail(FC_ERR_INVALID_ARG, "k_next / v_next overlap the current buffers or each other");
+  if (!(scale > 0.0f)) scale = 1.0f / sqrtf((float)d);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* w = static_cast<char*>(ws);
+  float* imp = reinterpret_cast<float*>(w + lay.imp);
+  float* red = reinterpret_cast<float*>(w + lay.red);
+  int32_t* sel = idx != nullptr ? idx : reinterpret_cast<int32_t*>(w + lay.idx);
+  const bool bf16 = dtype == FC_BF16;
+  cudaError_t e = (bf16 && fc::importance_tc_supported(d))
+                      ? fc::launch_importance_tc(q, k_buf, H, Lq, cap, d, scale, imp, w, s)
+                      : fc::launch_importance_simt(q, k_buf, bf16, H, Lq, cap, d, scale, imp, w, s);
+  if (e == cudaSuccess) e = fc::launch_redundancy(k_buf, bf16, H, cap, d, red, w + lay.red_ws, s);
+  if (e == cudaSuccess)
+    e = fc::launch_score_topb(imp, red, H, cap, pool_window, lambda, B_budget, nullptr, sel,
+                              w + lay.score_ws, s);
+  if (e == cudaSuccess)
+    e = fc::launch_compact(k_buf, v_buf, (int)elem_bytes(dtype), H, cap, d, sel, B_budget, cap,
+                           k_next, v_next, s);
+  st = launched(e, "fc_kv_cache_commit");
+  if (st == FC_OK) {
+    *n_next = B_budget;
+    *compressed = 1;
+  }
+  return st;
 }
 
 fc_status fc_selftest_exp2(const float* x, float* y_mufu, float* y_poly, int n, void* stream) {

@@ -31,6 +31,9 @@ __all__ = [
     "KVConfig",
     "GateConfig",
     "KV_CONFIGS",
+    "CacheConfig",
+    "CACHE_CONFIGS",
+    "cache_inputs",
     "GATE_CONFIGS",
     "kv_inputs",
     "kv_head",
@@ -121,6 +124,34 @@ GATE_CONFIGS = {
                                   m=5, eps=(0.01,), kind="toy", p=2.0,
                                   x0_std=tuple(0.05 * (1 + (c % 4)) for c in range(16)),
                                   stagger=3, latent_shape=(24, 45, 45, 16)),
+}
+
+
+@dataclass(frozen=True)
+class CacheConfig:
+    """A stream of chunks entering the fixed KV buffer B_budget + C per head:
+    C tokens per chunk, L_q queries of the chunk denoising at each commit."""
+
+    name: str
+    H: int
+    d: int
+    C: int
+    B_budget: int
+    n_chunks: int
+    Lq: int
+    lam: float
+    pool: int
+    dtype: str
+    rho: float
+
+
+CACHE_CONFIGS = {
+    # 2 heads, d=64, chunks of 48 tokens, budget 2 chunks, 6 chunks, float32.
+    "tiny_fp32_stream": CacheConfig("tiny_fp32_stream", H=2, d=64, C=48, B_budget=96,
+                                    n_chunks=6, Lq=40, lam=0.5, pool=3, dtype="f32", rho=0.9),
+    # 4 heads, d=128, chunks of 1024 tokens, budget 4 chunks, 8 chunks, bf16.
+    "bf16_stream": CacheConfig("bf16_stream", H=4, d=128, C=1024, B_budget=4096, n_chunks=8,
+                               Lq=256, lam=0.5, pool=7, dtype="bf16", rho=0.95),
 }
 
 
@@ -272,3 +303,19 @@ def gate_dt(cfg: GateConfig, steps):
         else:
             dt[c] = -1.0 / cfg.T
     return dt
+
+
+def cache_inputs(cfg: CacheConfig, seed=0):
+    """Chunk K and V ([n_chunks] of [H, C, d]) and, per chunk, the queries of
+    the chunk denoising when it finishes ([n_chunks] of [H, L_q, d]), torch
+    CPU tensors.  The keys are one AR(1) walk across the whole stream, cut into
+    chunks, so consecutive chunks are correlated as video tokens are."""
+    kv = KVConfig(cfg.name, H=cfg.H, d=cfg.d, Lq=cfg.Lq * cfg.n_chunks, Lk=cfg.C * cfg.n_chunks,
+                  B=cfg.B_budget, lam=(cfg.lam,), pool=cfg.pool, dtype=cfg.dtype, rho=cfg.rho)
+    Q, K, V = kv_inputs(kv, seed=seed)
+    C, Lq = cfg.C, cfg.Lq
+    ks = [K[:, i * C:(i + 1) * C].contiguous() for i in range(cfg.n_chunks)]
+    vs = [V[:, i * C:(i + 1) * C].contiguous() for i in range(cfg.n_chunks)]
+    qs = [Q[:, i * Lq:(i + 1) * Lq].contiguous() for i in range(cfg.n_chunks)]
+    return ks, vs, qs
+

@@ -298,6 +298,59 @@ fc_status fc_kv_score_topb(const float* imp, const float* red, int H, int Lk, in
 fc_status fc_kv_compact(const void* k, const void* v, fc_dtype dtype, int H, int Lk, int d,
                         const int32_t* idx, int B, void* k_out, void* v_out, void* stream);
 
+/* ------------------------------------------------------------------------ */
+/* Cache buffer management around compression (key design 3 and the         */
+/* flowchart: finished chunks enter the KV cache; when the reserved cache  */
+/* is full the new chunk is merged and every head keeps its top-B tokens)  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Bytes of workspace fc_kv_cache_commit needs (0 for invalid sizes).
+ * Bytes 0..3 of that workspace are the importance stage's error word, with
+ * the meaning and zero-initialisation rule of fc_kv_importance's.
+ */
+size_t fc_kv_cache_workspace_size(fc_dtype dtype, int H, int Lq, int B_budget, int C, int d);
+
+/*
+ * One chunk that has finished denoising enters the cache.
+ *
+ * The fixed buffer per head holds cap = B_budget + C rows: rows [0, n_clean)
+ * are the compressed clean tokens, rows [n_clean, n_clean + C) the chunk that
+ * just finished (the denoising forward wrote its K/V there, so the merge
+ * moves nothing).
+ *   - If n_clean + C <= B_budget the chunk is kept where it is: *n_next =
+ *     n_clean + C, *compressed = 0, nothing is launched and no device pointer
+ *     is read (they may be NULL).
+ *   - Otherwise the cap candidates are scored as fc_kv_importance (queries q),
+ *     fc_kv_redundancy and fc_kv_score_topb with B = B_budget would score them,
+ *     and the kept rows of every head are written once, in candidate order, to
+ *     rows [0, B_budget) of the other buffer (k_next, v_next); rows
+ *     [B_budget, cap) of that buffer are not written (the next chunk's K/V go
+ *     there).  *n_next = B_budget, *compressed = 1: the caller swaps buffers.
+ *
+ *   q              [H][Lq][d] dtype, queries of the chunk now denoising
+ *   k_buf, v_buf   [H][cap][d] dtype, the current buffer (read only)
+ *   k_next, v_next [H][cap][d] dtype, the other buffer; no overlap with the
+ *                  current one or with each other
+ *   d              64 or 128
+ *   C              tokens per chunk, >= 1; B_budget a multiple of C (so a
+ *                  compression always sees exactly cap candidates)
+ *   n_clean        a multiple of C in [0, B_budget]
+ *   scale          softmax scale, <= 0 means 1/sqrt(d)
+ *   pool_window, lambda  as for fc_kv_score_topb
+ *   idx            [H][B_budget] int32 out (the kept candidate rows,
+ *                  ascending), or NULL to keep them in the workspace only
+ *   n_next, compressed   host ints, out
+ * Errors: bad sizes or pointers, overlapping buffers -> FC_ERR_INVALID_ARG;
+ * B_budget not a multiple of C, d not 64/128 -> FC_ERR_UNSUPPORTED; small
+ * ws -> FC_ERR_WORKSPACE.  On an error *n_next and *compressed are unchanged.
+ */
+fc_status fc_kv_cache_commit(const void* q, const void* k_buf, const void* v_buf, void* k_next,
+                             void* v_next, fc_dtype dtype, int H, int Lq, int d, int B_budget,
+                             int C, int n_clean, float scale, int pool_window, float lambda,
+                             int32_t* idx, void* ws, size_t ws_bytes, int* n_next,
+                             int* compressed, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -143,3 +143,41 @@ def test_mask_consumer_validates_on_the_host():
     assert lib.fc_last_error() == b"x is NULL"
     assert lib.fc_scatter_velocity(NULL, NULL, NULL, 4, 8, NULL, NULL) == 1
     assert lib.fc_last_error() == b"v_dense is NULL"
+
+
+def test_cache_commit_validates_and_keeps_fitting_chunks_on_the_host():
+    lib = fc.library()
+    n_next, comp = ctypes.c_int(-1), ctypes.c_int(-1)
+    ref = (ctypes.byref(n_next), ctypes.byref(comp))
+
+    host = ctypes.create_string_buffer(256)
+
+    def commit(dtype=fc.FC_BF16, H=2, Lq=8, d=64, B=96, C=32, n=0, pool=3, ws_bytes=0):
+        ws = ctypes.addressof(host) if ws_bytes else NULL
+        return lib.fc_kv_cache_commit(NULL, NULL, NULL, NULL, NULL, dtype, H, Lq, d, B, C, n,
+                                      0.0, pool, 0.5, NULL, ws, ws_bytes, *ref, NULL)
+
+    # the chunk fits: nothing is launched and no device pointer is needed
+    assert commit(n=64) == 0 and (n_next.value, comp.value) == (96, 0)
+    assert lib.fc_last_launches() == 0
+    n_next.value = comp.value = -1
+    assert commit(B=96, C=96, n=0) == 0 and (n_next.value, comp.value) == (96, 0)
+    # B_budget not a multiple of C; d unsupported
+    assert commit(B=100, C=32) == 2
+    assert commit(d=96) == 2
+    # n_clean not a multiple of C, out of range, C < 1, C > B_budget, even window
+    assert commit(n=16) == 1
+    assert commit(n=128) == 1
+    assert commit(C=0) == 1
+    assert commit(C=128) == 1
+    assert commit(n=64, pool=4) == 1
+    # a full cache needs the workspace
+    assert commit(n=96) == 3
+    assert b"workspace" in lib.fc_last_error()
+    # the error paths leave the outputs alone
+    n_next.value = comp.value = -1
+    assert commit(n=96, ws_bytes=1 << 30) == 1  # then the NULL q (ws is never read here)
+    assert lib.fc_last_error() == b"q is NULL"
+    assert (n_next.value, comp.value) == (-1, -1)
+    assert lib.fc_kv_cache_workspace_size(fc.FC_BF16, 2, 8, 96, 32, 64) > 0
+    assert lib.fc_kv_cache_workspace_size(fc.FC_BF16, 2, 8, 96, 32, 96) == 0
