@@ -12,10 +12,14 @@ lambda=0.5, pool 7) with the gate over 4 chunks of 24x45x45x16 fp32 latents
 
 Metric: clean KV tokens scored+selected per second per head (= L_k / step
 time, summed over ranks); the gate's GB/s and each kernel's roofline fraction
-ride along.  Multi-GPU: every rank runs an independent layer (weak scaling,
-no data-path collective); timing is the max over ranks.
+ride along.  Multi-GPU (timing is the max over ranks, no data-path collective):
+  --shard layers (default)  every rank runs an independent layer (weak scaling);
+  --shard heads             one layer's heads, and the gate's chunks, are split
+                            over the ranks (strong scaling: every head and every
+                            chunk is independent, so nothing is exchanged).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
+                    [--workload NAME] [--shard layers|heads]
 """
 
 import argparse
@@ -52,6 +56,7 @@ def _args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="bf16_layer")
+    ap.add_argument("--shard", default="layers", choices=["layers", "heads"])
     ap.add_argument("--cpu-sample-heads", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -121,40 +126,66 @@ class Clocks:
 # ---------------------------------------------------------------------------
 # native arm
 # ---------------------------------------------------------------------------
-class Step:
-    """Device buffers of one layer's step and the five C-ABI calls."""
+def configs(workload):
+    """(KV workload, gate workload or None) of a bench workload name: the
+    full-step sweep layers share the 16-chunk gate; the long-history layer
+    has no gate."""
+    from cache_gating_kv_b200 import workloads as W
 
-    def __init__(self, kv_cfg, gate_cfg, seed, dev):
+    kv_cfg = W.KV_CONFIGS[workload]
+    if workload in W.GATE_CONFIGS:
+        return kv_cfg, W.GATE_CONFIGS[workload]
+    if workload.startswith("sweep_lk"):
+        return kv_cfg, W.GATE_CONFIGS["full_step_sweep"]
+    return kv_cfg, None
+
+
+class Step:
+    """Device buffers of one step and the five C-ABI calls.  ``heads`` and
+    ``chunks`` ([lo, hi) ranges) select this rank's share of the layer's heads
+    and of the gate's chunks; by default the whole layer."""
+
+    def __init__(self, kv_cfg, gate_cfg, seed, dev, heads=None, chunks=None):
         import cache_gating_kv_b200 as fc
         from cache_gating_kv_b200 import workloads as W
 
         self.fc = fc
         self.kv, self.gc = kv_cfg, gate_cfg
-        q, k, v = W.kv_inputs(kv_cfg, seed=seed)
+        q, k, v = W.kv_inputs(kv_cfg, seed=seed,
+                              heads=None if heads is None else range(*heads))
         self.host = {"q": q, "k": k, "v": v}
-        x = W.gate_initial(gate_cfg, seed)
-        vel = W.gate_velocity(gate_cfg, seed)
-        gstep = gate_cfg.m + 5 + gate_cfg.stagger * (gate_cfg.n_chunks - 1)
-        st = W.gate_step_counters(gate_cfg, min(gstep, gate_cfg.T - 1))
-        dt = W.gate_dt(gate_cfg, st)
-        self.host.update(x=torch.from_numpy(x), vel=torch.from_numpy(vel),
-                         dt=torch.from_numpy(dt), step=torch.from_numpy(st),
-                         f=torch.zeros(gate_cfg.n_chunks))
+        n_c = 0
+        if gate_cfg is not None:
+            x = W.gate_initial(gate_cfg, seed)
+            vel = W.gate_velocity(gate_cfg, seed)
+            gstep = gate_cfg.m + 5 + gate_cfg.stagger * (gate_cfg.n_chunks - 1)
+            st = W.gate_step_counters(gate_cfg, min(gstep, gate_cfg.T - 1))
+            dt = W.gate_dt(gate_cfg, st)
+            lo, hi = (0, gate_cfg.n_chunks) if chunks is None else chunks
+            n_c = hi - lo
+            if n_c > 0:
+                self.host.update(x=torch.from_numpy(x[lo:hi].copy()),
+                                 vel=torch.from_numpy(vel[lo:hi].copy()),
+                                 dt=torch.from_numpy(dt[lo:hi].copy()),
+                                 step=torch.from_numpy(st[lo:hi].copy()), f=torch.zeros(n_c))
+        self.n_c = n_c
         self.d = {n: t.to(dev) for n, t in self.host.items()}
-        H, Lq, Lk, d, B = kv_cfg.H, kv_cfg.Lq, kv_cfg.Lk, kv_cfg.d, kv_cfg.B
+        H = q.shape[0]
+        self.H = H
+        Lq, Lk, d, B = kv_cfg.Lq, kv_cfg.Lk, kv_cfg.d, kv_cfg.B
         code = fc.FC_BF16 if kv_cfg.dtype == "bf16" else fc.FC_F32
-        self.eps = gate_cfg.eps[0]
+        self.eps = gate_cfg.eps[0] if gate_cfg is not None else None
         self.lam = kv_cfg.lam[len(kv_cfg.lam) // 2]
         self.out = {
-            "l1": torch.zeros(gate_cfg.n_chunks, device=dev),
-            "mask": torch.zeros(gate_cfg.n_chunks, dtype=torch.uint8, device=dev),
+            "l1": torch.zeros(max(n_c, 1), device=dev),
+            "mask": torch.zeros(max(n_c, 1), dtype=torch.uint8, device=dev),
             "imp": torch.empty(H, Lk, device=dev), "red": torch.empty(H, Lk, device=dev),
             "idx": torch.empty(H, B, dtype=torch.int32, device=dev),
             "ko": torch.empty(H, B, d, dtype=q.dtype, device=dev),
             "vo": torch.empty(H, B, d, dtype=q.dtype, device=dev),
         }
         self.ws = {
-            "gate": fc.workspace(fc.fc_gate_workspace_size(gate_cfg.n_chunks, gate_cfg.N), dev),
+            "gate": fc.workspace(fc.fc_gate_workspace_size(n_c, gate_cfg.N) if n_c else 256, dev),
             "imp": fc.workspace(fc.fc_importance_workspace_size(code, H, Lq, Lk, d), dev),
             "red": fc.workspace(fc.fc_redundancy_workspace_size(code, H, Lk, d), dev),
             "topb": fc.workspace(fc.fc_score_topb_workspace_size(H, Lk, B), dev),
@@ -167,9 +198,10 @@ class Step:
         n = 0
         if ev:
             ev[0].record(stream)
-        fc.fc_chunk_l1_gate(d["x"], d["vel"], d["dt"], d["step"], self.gc.m, self.eps, d["f"],
-                            o["l1"], o["mask"], w["gate"], stream=stream)
-        n += fc.fc_last_launches()
+        if self.n_c:
+            fc.fc_chunk_l1_gate(d["x"], d["vel"], d["dt"], d["step"], self.gc.m, self.eps,
+                                d["f"], o["l1"], o["mask"], w["gate"], stream=stream)
+            n += fc.fc_last_launches()
         if ev:
             ev[1].record(stream)
         fc.fc_kv_importance(d["q"], d["k"], o["imp"], w["imp"], stream=stream)
@@ -192,8 +224,9 @@ class Step:
         return n
 
     def reset_gate(self):
-        self.d["x"].copy_(self.host["x"])
-        self.d["f"].zero_()
+        if self.n_c:
+            self.d["x"].copy_(self.host["x"])
+            self.d["f"].zero_()
 
 
 def reduce_max(values, world, device):
@@ -222,8 +255,19 @@ def native(a, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    kv_cfg, gate_cfg = W.KV_CONFIGS[a.workload], W.GATE_CONFIGS[a.workload]
-    step = Step(kv_cfg, gate_cfg, seed=rank, dev=dev)
+    kv_cfg, gate_cfg = configs(a.workload)
+    by_heads = a.shard == "heads" and world > 1
+    if by_heads:
+        if world > kv_cfg.H:
+            raise SystemExit(f"--shard heads needs at most H={kv_cfg.H} ranks")
+        heads = shard_heads(kv_cfg.H, rank, world)
+        chunks = shard_heads(gate_cfg.n_chunks, rank, world) if gate_cfg else None
+        step = Step(kv_cfg, gate_cfg, seed=0, dev=dev, heads=heads, chunks=chunks)
+        per_rank = (f"heads [{heads[0]}, {heads[1]}) of one layer"
+                    + (f", gate chunks [{chunks[0]}, {chunks[1]})" if chunks else ""))
+    else:
+        step = Step(kv_cfg, gate_cfg, seed=rank, dev=dev)
+        per_rank = "one independent layer per GPU"
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
@@ -273,6 +317,7 @@ def native(a, rank, world, local_rank):
         ck = clocks.stop()
         gate16 = _gate_alone(W.GATE_CONFIGS["full_step_sweep"], rank, dev, stream, flush, sink,
                              a.steps)
+        barrier()
     del graph
     ms_step = sum(tot) / len(tot)
     ms_call = {n: sum(v) / len(v) for n, v in per.items()}
@@ -286,12 +331,16 @@ def native(a, rank, world, local_rank):
     t_max = maxed[0]
     if e2e:
         e2e["ms"] = maxed[1]
-    H, Lq, Lk, d = kv_cfg.H, kv_cfg.Lq, kv_cfg.Lk, kv_cfg.d
-    value = world * Lk / (t_max * 1e-3)  # tokens/s per head over all ranks
+    H, Lq, Lk, d = step.H, kv_cfg.Lq, kv_cfg.Lk, kv_cfg.d
+    # tokens/s per head over all ranks: each rank finishes a layer per step (by
+    # layers), or all ranks together finish one layer per step (by heads)
+    layers = 1 if by_heads else world
+    value = layers * Lk / (t_max * 1e-3)
     hbm, tf_burst, tf_sus, src = _peaks()
     exec_flops = 4.0 * H * Lq * Lk * d  # two passes of Q K^T
     imp_tf = exec_flops / (ms_call["importance"] * 1e-3) / 1e12
-    gate_gbs = _bytes_gate(gate_cfg) / (ms_call["gate"] * 1e-3) / 1e9
+    gate_gbs = (_bytes_gate(gate_cfg) * step.n_c / gate_cfg.n_chunks / (ms_call["gate"] * 1e-3)
+                / 1e9) if step.n_c else None
     elem = 2 if kv_cfg.dtype == "bf16" else 4
     red_gbs = H * Lk * d * elem / (ms_call["redundancy"] * 1e-3) / 1e9
     comp_gbs = 2 * 2 * H * kv_cfg.B * d * elem / (ms_call["compact"] * 1e-3) / 1e9
@@ -299,13 +348,15 @@ def native(a, rank, world, local_rank):
     launches = launches_per_step * a.steps
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
-        "warmup": a.warmup, "ms_per_step": t_max, "higher_is_better": True, "scaling": "weak",
+        "warmup": a.warmup, "ms_per_step": t_max, "higher_is_better": True,
+        "scaling": "strong" if by_heads else "weak",
         "vs_baseline": None, "dtype": kv_cfg.dtype if kv_cfg.dtype == "bf16" else "f32",
         "data": "synthetic (seeded AR(1) keys, N(0,1) queries/values, flow-matching toy latents)",
-        "config": {"workload": f"{a.workload}: H={H} d={d} L_q={Lq} L_k={Lk} B={kv_cfg.B} "
-                               f"lambda={step.lam} pool={kv_cfg.pool}; gate {gate_cfg.n_chunks}x"
-                               f"{gate_cfg.N} fp32 m={gate_cfg.m} eps={step.eps}",
-                   "per_rank": "one independent layer per GPU",
+        "config": {"workload": f"{a.workload}: H={kv_cfg.H} d={d} L_q={Lq} L_k={Lk} "
+                               f"B={kv_cfg.B} lambda={step.lam} pool={kv_cfg.pool}; " +
+                               (f"gate {gate_cfg.n_chunks}x{gate_cfg.N} fp32 m={gate_cfg.m} "
+                                f"eps={step.eps}" if gate_cfg else "no gate"),
+                   "per_rank": per_rank,
                    "l2": "flushed between steps (256 MiB write + read-back, outside the timed "
                          "events)"},
         "roofline": {"bound": "tensor", "kernel": "fc_kv_importance (2 passes)",
@@ -317,7 +368,7 @@ def native(a, rank, world, local_rank):
                      "traffic": 263.2e6 if a.workload == "bf16_layer" else None,
                      "traffic_unit": "bytes per call"},
         "kernels_ms": ms_call,
-        "gate": {"GB/s": gate_gbs, "frac_hbm": gate_gbs / hbm},
+        "gate": {"GB/s": gate_gbs, "frac_hbm": gate_gbs / hbm if gate_gbs else None},
         "gate_full_step_sweep": {"chunks": 16, "us": gate16 * 1e3,
                                  "GB/s": _bytes_gate(W.GATE_CONFIGS["full_step_sweep"]) /
                                  (gate16 * 1e-3) / 1e9,
@@ -333,7 +384,7 @@ def native(a, rank, world, local_rank):
         "clocks": ck,
     }
     if e2e:
-        out["e2e"] = {"value": world * Lk / (e2e["ms"] * 1e-3), "unit": UNIT,
+        out["e2e"] = {"value": layers * Lk / (e2e["ms"] * 1e-3), "unit": UNIT,
                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
     return out
 
@@ -375,12 +426,13 @@ def _e2e(step, stream, flush, sink, a, dev):
     """Same step with pinned host inputs copied in and the results read back,
     inside the timed region, every step."""
     host_in = {n: t.pin_memory() for n, t in step.host.items()}
-    res = ["l1", "mask", "idx"]
+    res = (["l1", "mask"] if step.n_c else []) + ["idx"]
     host_out = {n: torch.empty_like(step.out[n], device="cpu").pin_memory() for n in res}
+    if step.n_c:
+        res.append("f")
+        host_out["f"] = torch.empty_like(step.host["f"]).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
-    d2h = sum(t.numel() * t.element_size() for t in host_out.values()) + \
-        step.d["f"].numel() * 4
-    host_f = torch.empty_like(step.host["f"]).pin_memory()
+    d2h = sum(t.numel() * t.element_size() for t in host_out.values())
     times = []
     with torch.cuda.stream(stream):
         for i in range(a.warmup + a.steps):
@@ -391,8 +443,7 @@ def _e2e(step, stream, flush, sink, a, dev):
                 step.d[n].copy_(t, non_blocking=True)
             step.run(stream)
             for n in res:
-                host_out[n].copy_(step.out[n], non_blocking=True)
-            host_f.copy_(step.d["f"], non_blocking=True)
+                host_out[n].copy_(step.d["f"] if n == "f" else step.out[n], non_blocking=True)
             e1.record(stream)
             e1.synchronize()
             if i >= a.warmup:
@@ -404,7 +455,8 @@ def _e2e(step, stream, flush, sink, a, dev):
 # CPU oracle legs
 # ---------------------------------------------------------------------------
 def _oracle_step_seconds(kv_cfg, gate_cfg, heads, seed=0):
-    """Oracle time for the compression of ``heads`` heads plus one full gate step."""
+    """Oracle time for the compression of ``heads`` heads plus one full gate
+    step (0 when the workload has no gate)."""
     from cache_gating_kv_b200 import workloads as W
     from oracle import flowcache_oracle as O
 
@@ -412,20 +464,23 @@ def _oracle_step_seconds(kv_cfg, gate_cfg, heads, seed=0):
     q64 = q.float().numpy().astype(np.float64)
     k64 = k.float().numpy().astype(np.float64)
     kf, vf = k.float().numpy(), v.float().numpy()
-    x = W.gate_initial(gate_cfg, seed)
-    vel = W.gate_velocity(gate_cfg, seed)
-    st = W.gate_step_counters(gate_cfg, gate_cfg.m + 5)
-    dt = W.gate_dt(gate_cfg, st)
     lam = kv_cfg.lam[len(kv_cfg.lam) // 2]
+    t_gate = 0.0
+    if gate_cfg is not None:
+        x = W.gate_initial(gate_cfg, seed)
+        vel = W.gate_velocity(gate_cfg, seed)
+        st = W.gate_step_counters(gate_cfg, gate_cfg.m + 5)
+        dt = W.gate_dt(gate_cfg, st)
+        t0 = time.perf_counter()
+        O.gate_step(x, vel, dt, st, gate_cfg.m, gate_cfg.eps[0],
+                    np.zeros(gate_cfg.n_chunks, np.float32))
+        t_gate = time.perf_counter() - t0
     t0 = time.perf_counter()
-    O.gate_step(x, vel, dt, st, gate_cfg.m, gate_cfg.eps[0], np.zeros(gate_cfg.n_chunks, np.float32))
-    t1 = time.perf_counter()
     imp = O.importance(q64, k64)
     red = O.redundancy(k64)
     _, idx = O.score_topb(imp, red, lam, kv_cfg.pool, kv_cfg.B)
     O.compact(kf, vf, idx)
-    t2 = time.perf_counter()
-    return t1 - t0, (t2 - t1) / heads
+    return t_gate, (time.perf_counter() - t0) / heads
 
 
 def _cores():
@@ -439,7 +494,7 @@ def _cores():
 def cpu_baseline(a):
     from cache_gating_kv_b200 import workloads as W
 
-    kv_cfg, gate_cfg = W.KV_CONFIGS[a.workload], W.GATE_CONFIGS[a.workload]
+    kv_cfg, gate_cfg = configs(a.workload)
     heads = max(1, min(a.cpu_sample_heads, kv_cfg.H))
     t_gate, t_head = _oracle_step_seconds(kv_cfg, gate_cfg, heads)
     t_step = t_gate + kv_cfg.H * t_head
@@ -454,7 +509,7 @@ def reference(a, rank):
         return None
     from cache_gating_kv_b200 import workloads as W
 
-    kv_cfg, gate_cfg = W.KV_CONFIGS[a.workload], W.GATE_CONFIGS[a.workload]
+    kv_cfg, gate_cfg = configs(a.workload)
     times = []
     for i in range(a.warmup + a.steps):
         t_gate, t_head = _oracle_step_seconds(kv_cfg, gate_cfg, 1, seed=i)
