@@ -57,6 +57,8 @@ def _args():
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="bf16_layer")
     ap.add_argument("--shard", default="layers", choices=["layers", "heads"])
+    ap.add_argument("--serial", action="store_true",
+                    help="run the five calls one after another on one stream")
     ap.add_argument("--cpu-sample-heads", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -184,6 +186,8 @@ class Step:
             "ko": torch.empty(H, B, d, dtype=q.dtype, device=dev),
             "vo": torch.empty(H, B, d, dtype=q.dtype, device=dev),
         }
+        self.fork = torch.cuda.Event()
+        self.join = torch.cuda.Event()
         self.ws = {
             "gate": fc.workspace(fc.fc_gate_workspace_size(n_c, gate_cfg.N) if n_c else 256, dev),
             "imp": fc.workspace(fc.fc_importance_workspace_size(code, H, Lq, Lk, d), dev),
@@ -191,36 +195,50 @@ class Step:
             "topb": fc.workspace(fc.fc_score_topb_workspace_size(H, Lk, B), dev),
         }
 
-    def run(self, stream, ev=None):
-        """Enqueue one step; ``ev`` (6 events) brackets the five calls.
-        Returns the number of kernel launches the library enqueued."""
+    # events bracketing the calls: call -> (start event, end event)
+    SPANS = {"gate": ("gate0", "gate1"), "redundancy": ("gate1", "red1"),
+             "importance": ("imp0", "imp1"), "score_topb": ("join", "score1"),
+             "compact": ("score1", "end")}
+    EVENTS = ("start", "gate0", "gate1", "red1", "imp0", "imp1", "join", "score1", "end")
+
+    def run(self, stream, ev=None, side=None):
+        """Enqueue one step; returns the number of kernel launches the library
+        enqueued.  The gate and the redundancy depend on nothing else in the
+        step, so with a ``side`` stream they run there, beside the importance
+        on ``stream``, and the score waits for both.  ``ev`` maps the names in
+        EVENTS to timing events."""
         fc, d, o, w = self.fc, self.d, self.out, self.ws
+        rec = (lambda k, st: ev[k].record(st)) if ev else (lambda k, st: None)
+        s2 = side if side is not None else stream
         n = 0
-        if ev:
-            ev[0].record(stream)
+        rec("start", stream)
+        if side is not None:
+            self.fork.record(stream)
+            side.wait_event(self.fork)
+        rec("gate0", s2)
         if self.n_c:
             fc.fc_chunk_l1_gate(d["x"], d["vel"], d["dt"], d["step"], self.gc.m, self.eps,
-                                d["f"], o["l1"], o["mask"], w["gate"], stream=stream)
+                                d["f"], o["l1"], o["mask"], w["gate"], stream=s2)
             n += fc.fc_last_launches()
-        if ev:
-            ev[1].record(stream)
+        rec("gate1", s2)
+        fc.fc_kv_redundancy(d["k"], o["red"], w["red"], stream=s2)
+        n += fc.fc_last_launches()
+        rec("red1", s2)
+        rec("imp0", stream)
         fc.fc_kv_importance(d["q"], d["k"], o["imp"], w["imp"], stream=stream)
         n += fc.fc_last_launches()
-        if ev:
-            ev[2].record(stream)
-        fc.fc_kv_redundancy(d["k"], o["red"], w["red"], stream=stream)
-        n += fc.fc_last_launches()
-        if ev:
-            ev[3].record(stream)
+        rec("imp1", stream)
+        if side is not None:
+            self.join.record(side)
+            stream.wait_event(self.join)
+        rec("join", stream)
         fc.fc_kv_score_topb(o["imp"], o["red"], self.kv.pool, self.lam, self.kv.B, o["idx"],
                             w["topb"], stream=stream)
         n += fc.fc_last_launches()
-        if ev:
-            ev[4].record(stream)
+        rec("score1", stream)
         fc.fc_kv_compact(d["k"], d["v"], o["idx"], o["ko"], o["vo"], stream=stream)
         n += fc.fc_last_launches()
-        if ev:
-            ev[5].record(stream)
+        rec("end", stream)
         return n
 
     def reset_gate(self):
@@ -268,37 +286,43 @@ def native(a, rank, world, local_rank):
     else:
         step = Step(kv_cfg, gate_cfg, seed=rank, dev=dev)
         per_rank = "one independent layer per GPU"
-    stream = torch.cuda.Stream(device=dev)
+    # the importance (on the critical path) gets the higher priority; the gate
+    # and the redundancy fill the SMs it leaves idle
+    lo, hi = torch.cuda.Stream.priority_range()
+    stream = torch.cuda.Stream(device=dev, priority=hi)
+    side = None if a.serial else torch.cuda.Stream(device=dev, priority=lo)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     sink = torch.empty((), dtype=torch.float32, device=dev)
-    names = ["gate", "importance", "redundancy", "score_topb", "compact"]
+    names = list(Step.SPANS)
 
     def barrier():
         if world > 1:
             torch.distributed.barrier()
 
+    def events(external):
+        return {k: torch.cuda.Event(enable_timing=True, external=external) for k in Step.EVENTS}
+
     # One step is captured once as a CUDA graph (with timing events as graph
     # nodes) and replayed: the GPU runs the step's launches back to back
     # instead of waiting on the host between small kernels.
-    ev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(6)]
+    ev = events(True)
     with torch.cuda.stream(stream):
         for _ in range(a.warmup):
             flush_l2(flush, sink)
-            step.run(stream)
-        stream.synchronize()
-        t0 = time.perf_counter()
-        eager_ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+            step.run(stream, side=side)
+        torch.cuda.synchronize()
+        eager_ev = events(False)
         flush_l2(flush, sink)
-        launches_per_step = step.run(stream, eager_ev)
-        stream.synchronize()
-        ms_eager = eager_ev[0].elapsed_time(eager_ev[5])
+        launches_per_step = step.run(stream, eager_ev, side=side)
+        torch.cuda.synchronize()
+        ms_eager = eager_ev["start"].elapsed_time(eager_ev["end"])
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=stream, capture_error_mode="relaxed"):
-            step.run(stream, ev)
+            step.run(stream, ev, side=side)
         for _ in range(2):
             flush_l2(flush, sink)
             graph.replay()
-        stream.synchronize()
+        torch.cuda.synchronize()
         clocks = Clocks(local_rank)
         barrier()
         torch.cuda.synchronize()
@@ -309,23 +333,39 @@ def native(a, rank, world, local_rank):
             flush_l2(flush, sink)  # between steps, outside the timed events
             graph.replay()
             stream.synchronize()
-            for j, n in enumerate(names):
-                per[n].append(ev[j].elapsed_time(ev[j + 1]))
-            tot.append(ev[0].elapsed_time(ev[5]))
+            for n, (e0, e1) in Step.SPANS.items():
+                per[n].append(ev[e0].elapsed_time(ev[e1]))
+            tot.append(ev["start"].elapsed_time(ev["end"]))
         torch.cuda.synchronize()
         barrier()
         ck = clocks.stop()
+        # each call alone (one stream, one after another) for its own roofline
+        alone = per
+        if side is not None:
+            g1 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g1, stream=stream, capture_error_mode="relaxed"):
+                step.run(stream, ev)
+            alone = {n: [] for n in names}
+            for i in range(a.steps + 2):
+                flush_l2(flush, sink)
+                g1.replay()
+                stream.synchronize()
+                if i >= 2:
+                    for n, (e0, e1) in Step.SPANS.items():
+                        alone[n].append(ev[e0].elapsed_time(ev[e1]))
+            del g1
         gate16 = _gate_alone(W.GATE_CONFIGS["full_step_sweep"], rank, dev, stream, flush, sink,
                              a.steps)
         barrier()
     del graph
     ms_step = sum(tot) / len(tot)
     ms_call = {n: sum(v) / len(v) for n, v in per.items()}
+    ms_alone = {n: sum(v) / len(v) for n, v in alone.items()}
 
     # end to end through the public API with host buffers (pinned), every step
     e2e = None
     if not a.no_e2e:
-        e2e = _e2e(step, stream, flush, sink, a, dev)
+        e2e = _e2e(step, stream, side, flush, sink, a, dev)
 
     maxed = reduce_max([ms_step] + ([e2e["ms"]] if e2e else []), world, dev)
     t_max = maxed[0]
@@ -339,12 +379,12 @@ def native(a, rank, world, local_rank):
     hbm, tf_burst, tf_sus, src = _peaks()
     exec_flops = 4.0 * H * Lq * Lk * d  # two passes of Q K^T
     imp_tf = exec_flops / (ms_call["importance"] * 1e-3) / 1e12
-    gate_gbs = (_bytes_gate(gate_cfg) * step.n_c / gate_cfg.n_chunks / (ms_call["gate"] * 1e-3)
+    gate_gbs = (_bytes_gate(gate_cfg) * step.n_c / gate_cfg.n_chunks / (ms_alone["gate"] * 1e-3)
                 / 1e9) if step.n_c else None
     elem = 2 if kv_cfg.dtype == "bf16" else 4
-    red_gbs = H * Lk * d * elem / (ms_call["redundancy"] * 1e-3) / 1e9
-    comp_gbs = 2 * 2 * H * kv_cfg.B * d * elem / (ms_call["compact"] * 1e-3) / 1e9
-    topb_gbs = H * Lk * 12 / (ms_call["score_topb"] * 1e-3) / 1e9
+    red_gbs = H * Lk * d * elem / (ms_alone["redundancy"] * 1e-3) / 1e9
+    comp_gbs = 2 * 2 * H * kv_cfg.B * d * elem / (ms_alone["compact"] * 1e-3) / 1e9
+    topb_gbs = H * Lk * 12 / (ms_alone["score_topb"] * 1e-3) / 1e9
     launches = launches_per_step * a.steps
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
@@ -368,6 +408,10 @@ def native(a, rank, world, local_rank):
                      "traffic": 263.2e6 if a.workload == "bf16_layer" else None,
                      "traffic_unit": "bytes per call"},
         "kernels_ms": ms_call,
+        "kernels_ms_alone": ms_alone,
+        "kernels_note": "kernels_ms: spans inside the timed step (gate and redundancy share "
+                        "the GPU with the importance there); kernels_ms_alone: the same calls "
+                        "one after another on one stream, which the GB/s figures use",
         "gate": {"GB/s": gate_gbs, "frac_hbm": gate_gbs / hbm if gate_gbs else None},
         "gate_full_step_sweep": {"chunks": 16, "us": gate16 * 1e3,
                                  "GB/s": _bytes_gate(W.GATE_CONFIGS["full_step_sweep"]) /
@@ -375,8 +419,10 @@ def native(a, rank, world, local_rank):
                                  "frac_hbm": _bytes_gate(W.GATE_CONFIGS["full_step_sweep"]) /
                                  (gate16 * 1e-3) / 1e9 / hbm},
         "timing": "one step captured as a CUDA graph, replayed per step; CUDA events are "
-                  "graph nodes around each call; eager (host-launched) step for reference: "
-                  f"{ms_eager:.3f} ms",
+                  "graph nodes around each call" +
+                  ("" if a.serial else "; gate and redundancy on a second, lower-priority "
+                   "stream beside the importance (they depend on nothing else in the step)") +
+                  f"; eager (host-launched) step for reference: {ms_eager:.3f} ms",
         "redundancy": {"GB/s": red_gbs, "frac_hbm": red_gbs / hbm},
         "score_topb": {"GB/s": topb_gbs},
         "compact": {"GB/s": comp_gbs, "frac_hbm": comp_gbs / hbm},
@@ -422,7 +468,7 @@ def _gate_alone(gc, seed, dev, stream, flush, sink, steps):
     return sum(times) / len(times)
 
 
-def _e2e(step, stream, flush, sink, a, dev):
+def _e2e(step, stream, side, flush, sink, a, dev):
     """Same step with pinned host inputs copied in and the results read back,
     inside the timed region, every step."""
     host_in = {n: t.pin_memory() for n, t in step.host.items()}
@@ -441,7 +487,7 @@ def _e2e(step, stream, flush, sink, a, dev):
             e0.record(stream)
             for n, t in host_in.items():
                 step.d[n].copy_(t, non_blocking=True)
-            step.run(stream)
+            step.run(stream, side=side)
             for n in res:
                 host_out[n].copy_(step.d["f"] if n == "f" else step.out[n], non_blocking=True)
             e1.record(stream)
