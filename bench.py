@@ -423,6 +423,10 @@ def native(a, rank, world, local_rank):
                   ("" if a.serial else "; gate and redundancy on a second, lower-priority "
                    "stream beside the importance (they depend on nothing else in the step)") +
                   f"; eager (host-launched) step for reference: {ms_eager:.3f} ms",
+        "importance": {"TFLOP/s executed": imp_tf, "TFLOP/s algorithmic": imp_tf / 2,
+                       "Gexp/s": 2.0 * H * Lq * Lk / (ms_call["importance"] * 1e-3) / 1e9,
+                       "note": "both passes recompute Q K^T (executed = 2 x algorithmic "
+                               "flops); 2 exponentials per score"},
         "redundancy": {"GB/s": red_gbs, "frac_hbm": red_gbs / hbm},
         "score_topb": {"GB/s": topb_gbs},
         "compact": {"GB/s": comp_gbs, "frac_hbm": comp_gbs / hbm},
