@@ -142,6 +142,16 @@ def configs(workload):
     return kv_cfg, None
 
 
+def workload_desc(workload):
+    """The workload's name and sizes, as both arms report them."""
+    kv_cfg, gate_cfg = configs(workload)
+    lam = kv_cfg.lam[len(kv_cfg.lam) // 2]
+    return (f"{workload}: H={kv_cfg.H} d={kv_cfg.d} L_q={kv_cfg.Lq} L_k={kv_cfg.Lk} "
+            f"B={kv_cfg.B} lambda={lam} pool={kv_cfg.pool}; " +
+            (f"gate {gate_cfg.n_chunks}x{gate_cfg.N} fp32 m={gate_cfg.m} eps={gate_cfg.eps[0]}"
+             if gate_cfg else "no gate"))
+
+
 class Step:
     """Device buffers of one step and the five C-ABI calls.  ``heads`` and
     ``chunks`` ([lo, hi) ranges) select this rank's share of the layer's heads
@@ -392,10 +402,7 @@ def native(a, rank, world, local_rank):
         "scaling": "strong" if by_heads else "weak",
         "vs_baseline": None, "dtype": kv_cfg.dtype if kv_cfg.dtype == "bf16" else "f32",
         "data": "synthetic (seeded AR(1) keys, N(0,1) queries/values, flow-matching toy latents)",
-        "config": {"workload": f"{a.workload}: H={kv_cfg.H} d={d} L_q={Lq} L_k={Lk} "
-                               f"B={kv_cfg.B} lambda={step.lam} pool={kv_cfg.pool}; " +
-                               (f"gate {gate_cfg.n_chunks}x{gate_cfg.N} fp32 m={gate_cfg.m} "
-                                f"eps={step.eps}" if gate_cfg else "no gate"),
+        "config": {"workload": workload_desc(a.workload),
                    "per_rank": per_rank,
                    "l2": "flushed between steps (256 MiB write + read-back, outside the timed "
                          "events)"},
@@ -573,7 +580,7 @@ def reference(a, rank):
             "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": t * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
-            "config": {"workload": a.workload},
+            "config": {"workload": workload_desc(a.workload)},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
