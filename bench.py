@@ -62,6 +62,8 @@ def _args():
     ap.add_argument("--cpu-sample-heads", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-next", action="store_true",
+                    help="skip the timings of the cache commit, mask consumer and history gate")
     return ap.parse_args()
 
 
@@ -366,6 +368,10 @@ def native(a, rank, world, local_rank):
             del g1
         gate16 = _gate_alone(W.GATE_CONFIGS["full_step_sweep"], rank, dev, stream, flush, sink,
                              a.steps)
+        nxt = None
+        if not a.no_next:
+            hbm0, tf0, _, _ = _peaks()
+            nxt = _next_rows(step, dev, stream, flush, sink, max(3, min(a.steps, 10)), hbm0, tf0)
         barrier()
     del graph
     ms_step = sum(tot) / len(tot)
@@ -420,6 +426,7 @@ def native(a, rank, world, local_rank):
                         "the GPU with the importance there); kernels_ms_alone: the same calls "
                         "one after another on one stream, which the GB/s figures use",
         "gate": {"GB/s": gate_gbs, "frac_hbm": gate_gbs / hbm if gate_gbs else None},
+        "next_rows": nxt,
         "gate_full_step_sweep": {"chunks": 16, "us": gate16 * 1e3,
                                  "GB/s": _bytes_gate(W.GATE_CONFIGS["full_step_sweep"]) /
                                  (gate16 * 1e-3) / 1e9,
@@ -444,6 +451,93 @@ def native(a, rank, world, local_rank):
         out["e2e"] = {"value": layers * Lk / (e2e["ms"] * 1e-3), "unit": UNIT,
                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
     return out
+
+
+def _graph_ms(fn, stream, flush, sink, steps, warm=3):
+    """Mean CUDA-graph-timed duration (ms) of ``fn`` enqueued on ``stream``,
+    with L2 flushed before every replay."""
+    with torch.cuda.stream(stream):
+        fn()
+        stream.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True, external=True)
+        e1 = torch.cuda.Event(enable_timing=True, external=True)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="relaxed"):
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+        times = []
+        for i in range(steps + warm):
+            flush_l2(flush, sink)
+            g.replay()
+            stream.synchronize()
+            if i >= warm:
+                times.append(e0.elapsed_time(e1))
+        del g
+    return sum(times) / len(times)
+
+
+def _next_rows(step, dev, stream, flush, sink, steps, hbm, tf_peak):
+    """The rows built beyond the per-step path, each timed alone: the mask
+    consumer and the history-guided gate on the 16-chunk full-step-sweep
+    latents, and one cache commit that compresses a full one-layer buffer."""
+    import cache_gating_kv_b200 as fc
+    from cache_gating_kv_b200 import workloads as W
+
+    gc = W.GATE_CONFIGS["full_step_sweep"]
+    n_c, N = gc.n_chunks, gc.N
+    x = torch.from_numpy(W.gate_initial(gc, 0)).to(dev)
+    v = torch.from_numpy(W.gate_velocity(gc, 0)).to(dev)
+    mask = torch.zeros(n_c, dtype=torch.uint8, device=dev)
+    mask[::2] = 1  # half the chunks recompute
+    n_re = int(mask.sum().item())
+    dense = torch.empty_like(x)
+    ids = torch.empty(n_c, dtype=torch.int32, device=dev)
+    cnt = torch.empty(1, dtype=torch.int32, device=dev)
+    v_cache = v.clone()
+    ms_g = _graph_ms(lambda: fc.fc_gather_recompute(x, mask, dense, ids, cnt, stream=stream),
+                     stream, flush, sink, steps)
+    ms_s = _graph_ms(lambda: fc.fc_scatter_velocity(dense, ids, cnt, v_cache, stream=stream),
+                     stream, flush, sink, steps)
+    moved = 2 * n_re * N * 4
+    h_new = x.clone()
+    h_old = x + 0.01 * v
+    st = torch.full((n_c,), gc.m + 3, dtype=torch.int32, device=dev)
+    f = torch.zeros(n_c, device=dev)
+    dd = torch.empty(n_c, device=dev)
+    rf = torch.empty(n_c, dtype=torch.uint8, device=dev)
+    ws = fc.workspace(fc.fc_gate_workspace_size(n_c, N), dev)
+    ms_h = _graph_ms(lambda: fc.fc_history_l1_gate(h_old, h_new, st, gc.m, 0.05, f, dd, rf, ws,
+                                                   stream=stream), stream, flush, sink, steps)
+    del x, v, dense, v_cache, h_new, h_old
+    # one compression of a full cache: the step's layer as the buffer, C = L_k / 4
+    kv = step.kv
+    H, Lq, Lk, d = step.H, kv.Lq, kv.Lk, kv.d
+    C, Bb = Lk // 4, Lk - Lk // 4
+    qd, kb, vb = step.d["q"], step.d["k"], step.d["v"]
+    kn, vn = torch.empty_like(kb), torch.empty_like(vb)
+    code = fc.FC_BF16 if kb.dtype == torch.bfloat16 else fc.FC_F32
+    cws = fc.workspace(fc.fc_kv_cache_workspace_size(code, H, Lq, Bb, C, d), dev)
+    ms_c = _graph_ms(lambda: fc.fc_kv_cache_commit(qd, kb, vb, kn, vn, Bb, C, cws, kv.pool,
+                                                   0.5, stream=stream),
+                     stream, flush, sink, steps)
+    imp_flops = 4.0 * H * Lq * Lk * d
+    return {
+        "gather_recompute": {"us": ms_g * 1e3, "GB/s": moved / (ms_g * 1e-3) / 1e9,
+                             "frac_hbm": moved / (ms_g * 1e-3) / 1e9 / hbm,
+                             "workload": f"{n_re} of {n_c} chunks x {N} fp32"},
+        "scatter_velocity": {"us": ms_s * 1e3, "GB/s": moved / (ms_s * 1e-3) / 1e9,
+                             "frac_hbm": moved / (ms_s * 1e-3) / 1e9 / hbm,
+                             "workload": f"{n_re} of {n_c} chunks x {N} fp32"},
+        "history_gate": {"us": ms_h * 1e3, "GB/s": _bytes_gate(gc) / (ms_h * 1e-3) / 1e9,
+                         "frac_hbm": _bytes_gate(gc) / (ms_h * 1e-3) / 1e9 / hbm,
+                         "workload": f"{n_c} segments x {N} fp32"},
+        "cache_commit": {"ms": ms_c, "TFLOP/s importance-executed per commit":
+                         imp_flops / (ms_c * 1e-3) / 1e12,
+                         "frac_bf16": imp_flops / (ms_c * 1e-3) / 1e12 / tf_peak,
+                         "workload": f"H={H} d={d} L_q={Lq} C={C} B_budget={Bb} (a full "
+                                     f"buffer of B_budget + C candidates, {kv.dtype})"},
+    }
 
 
 def _gate_alone(gc, seed, dev, stream, flush, sink, steps):
