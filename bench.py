@@ -52,7 +52,7 @@ def flush_l2(buf, sink):
 def _args():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="bf16_layer")
@@ -78,29 +78,75 @@ def _peaks():
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+    """SM clocks and clock-event (throttle) reasons sampled during timing.
+
+    NVML is polled from a background thread every ~2 ms (only reads: nothing
+    about the GPU is changed); without NVML, nvidia-smi is polled every 100 ms.
+    The device is found by its PCI bus id, so that a remapped
+    CUDA_VISIBLE_DEVICES still samples the GPU the rank runs on."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index):
-        self.gpu = gpu_index
+    def __init__(self, device):
+        p = torch.cuda.get_device_properties(device)
+        self.bus = f"{p.pci_domain_id:08x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
         self.proc = None
+        self.thread = None
+        self.samples = []
         self.path = f"/tmp/fc_clocks_{os.getpid()}.csv"
 
+    def _nvml_loop(self, nv, handle, bits):
+        while not self.stop_flag:
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(handle, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(handle)
+                self.samples.append((mhz, [n for n, bit in bits if reasons & bit]))
+            except Exception:
+                pass
+            time.sleep(0.002)
+
     def start(self):
+        self.samples = []
+        self.stop_flag = False
+        try:
+            import threading
+
+            import pynvml as nv
+            nv.nvmlInit()
+            handle = nv.nvmlDeviceGetHandleByPciBusId(self.bus)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(handle, nv.NVML_CLOCK_SM)
+            bits = [("hw_slowdown", nv.nvmlClocksEventReasonHwSlowdown),
+                    ("hw_thermal_slowdown", nv.nvmlClocksEventReasonHwThermalSlowdown),
+                    ("sw_thermal_slowdown", nv.nvmlClocksEventReasonSwThermalSlowdown),
+                    ("sw_power_cap", nv.nvmlClocksEventReasonSwPowerCap),
+                    ("hw_power_brake", nv.nvmlClocksEventReasonHwPowerBrakeSlowdown)]
+            self.thread = threading.Thread(target=self._nvml_loop, args=(nv, handle, bits),
+                                           daemon=True)
+            self.thread.start()
+            time.sleep(0.01)
+            return
+        except Exception:
+            self.thread = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.gpu), "-lms", "100"],
+                 "-i", self.bus, "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
         except Exception:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
+            return self._summary([m for m, _ in self.samples], self.max_mhz,
+                                 sorted({r for _, rs in self.samples for r in rs}), "nvml")
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no clock sampler"]}
         time.sleep(0.25)
         self.proc.terminate()
         try:
@@ -116,15 +162,19 @@ class Clocks:
             os.remove(self.path)
         except OSError:
             pass
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
         mhz = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
         mx = max((float(r[2]) for r in rows if r[2].replace(".", "").isdigit()), default=None)
+        reasons = sorted({self.NAMES[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        return self._summary(mhz, mx, reasons, "nvidia-smi")
+
+    @staticmethod
+    def _summary(mhz, mx, reasons, source):
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": ["no samples"],
+                    "source": source}
         loaded = [m for m in mhz if mx and m > 0.5 * mx] or mhz
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
-        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": mx,
-                "reasons": reasons, "samples": len(rows)}
+        return {"sm_mhz": statistics.median(loaded), "sm_min_mhz": min(mhz), "sm_max_mhz": mx,
+                "reasons": reasons, "samples": len(mhz), "source": source}
 
 
 # ---------------------------------------------------------------------------
@@ -335,7 +385,7 @@ def native(a, rank, world, local_rank):
             flush_l2(flush, sink)
             graph.replay()
         torch.cuda.synchronize()
-        clocks = Clocks(local_rank)
+        clocks = Clocks(dev)
         barrier()
         torch.cuda.synchronize()
         clocks.start()
