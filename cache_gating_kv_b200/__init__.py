@@ -29,6 +29,11 @@ __all__ = [
     "fc_gather_recompute",
     "fc_scatter_velocity",
     "fc_kv_cache_workspace_size",
+    "fc_check_workspace",
+    "FC_WS_GATE",
+    "FC_WS_GATE_NOALLOC",
+    "FC_WS_IMPORTANCE",
+    "FC_WS_CACHE",
     "fc_kv_cache_commit",
     "fc_kv_importance",
     "fc_kv_redundancy",
@@ -84,6 +89,7 @@ def _declare(lib):
         "fc_kv_compact": (c_int, [c_p, c_p, c_int, c_int, c_int, c_int, c_p, c_int, c_p, c_p,
                                   c_p]),
         "fc_kv_cache_workspace_size": (c_sz, [c_int, c_int, c_int, c_int, c_int, c_int]),
+        "fc_check_workspace": (c_int, [c_int, c_p, c_int, c_int, c_p]),
         "fc_kv_cache_commit": (c_int, [c_p, c_p, c_p, c_p, c_p, c_int, c_int, c_int, c_int, c_int,
                                        c_int, c_int, c_f, c_int, c_f, c_p, c_p, c_sz,
                                        ctypes.POINTER(c_int), ctypes.POINTER(c_int), c_p]),
@@ -168,6 +174,21 @@ def fc_score_topb_workspace_size(H, Lk, B):
 
 def fc_kv_cache_workspace_size(dtype, H, Lq, B_budget, C, d):
     return library().fc_kv_cache_workspace_size(dtype, H, Lq, B_budget, C, d)
+
+
+FC_WS_GATE, FC_WS_GATE_NOALLOC, FC_WS_IMPORTANCE, FC_WS_CACHE = 0, 1, 2, 3
+
+
+def fc_check_workspace(kind, ws=None, n_chunks=0, clear=False, stream=None):
+    """True if no bounded device-side wait of the calls that used ``ws`` gave
+    up (synchronises the stream); False if one did (their outputs are not
+    valid).  ``clear`` resets the error word after reading it."""
+    st = library().fc_check_workspace(int(kind), _p(ws), int(n_chunks), 1 if clear else 0,
+                                      _s(stream))
+    if st == 5:
+        return False
+    _check("fc_check_workspace", st)
+    return True
 
 
 def workspace(nbytes, device=None):

@@ -19,6 +19,8 @@ cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t n_per_ch
 // Same kernel with its scratch in a static device array (no allocation, at
 // most gate_noalloc_max_chunks() chunks; calls must not overlap on the GPU).
 int gate_noalloc_max_chunks();
+// Device address of the no-alloc gate's static scratch on the current device.
+cudaError_t gate_noalloc_scratch(void** out);
 cudaError_t launch_gate_noalloc(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
                                 const float* dt, const int32_t* step, int m, float eps, float* f,
                                 float* l1, uint8_t* mask, cudaStream_t s);

@@ -245,6 +245,50 @@ fc_status fc_scatter_velocity(const float* v_dense, const int32_t* ids, const in
                   "fc_scatter_velocity");
 }
 
+fc_status fc_check_workspace(fc_ws_kind kind, const void* ws, int n_chunks, int clear,
+                             void* stream) {
+  fc::g_launches = 0;
+  size_t off = 0;
+  const char* base = static_cast<const char*>(ws);
+  switch (kind) {
+    case FC_WS_GATE:
+      if (n_chunks < 1) return fail(FC_ERR_INVALID_ARG, "n_chunks must be >= 1");
+      FC_CHECK_PTR(ws);
+      off = (size_t)n_chunks * sizeof(unsigned);
+      break;
+    case FC_WS_GATE_NOALLOC: {
+      if (n_chunks < 1 || n_chunks > fc::gate_noalloc_max_chunks())
+        return fail(FC_ERR_INVALID_ARG, "n_chunks must be in [1, %d]",
+                    fc::gate_noalloc_max_chunks());
+      void* p = nullptr;
+      const cudaError_t e = fc::gate_noalloc_scratch(&p);
+      if (e != cudaSuccess) return fail(FC_ERR_CUDA, "scratch address: %s", cudaGetErrorString(e));
+      base = static_cast<const char*>(p);
+      off = (size_t)n_chunks * sizeof(unsigned);
+      break;
+    }
+    case FC_WS_IMPORTANCE:
+    case FC_WS_CACHE:
+      FC_CHECK_PTR(ws);
+      break;
+    default:
+      return fail(FC_ERR_INVALID_ARG, "unknown workspace kind %d", (int)kind);
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int word = 0;
+  cudaError_t e = cudaMemcpyAsync(&word, base + off, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e == cudaSuccess && clear && word != 0) {
+    e = cudaMemsetAsync(const_cast<char*>(base) + off, 0, sizeof(int), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  }
+  if (e != cudaSuccess) return fail(FC_ERR_CUDA, "reading the error word: %s", cudaGetErrorString(e));
+  if (word != 0)
+    return fail(FC_ERR_TIMEOUT, "a bounded device-side wait gave up: the outputs of the "
+                                "calls since the word was last clear are not valid");
+  return ok();
+}
+
 size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d) {
   (void)dtype;
   (void)Lk;

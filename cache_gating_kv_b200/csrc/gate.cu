@@ -392,10 +392,7 @@ void* g_gate_scratch_addr[128] = {nullptr};
 
 int gate_noalloc_max_chunks() { return kGateNoAllocMaxChunks; }
 
-cudaError_t launch_gate_noalloc(float* x, const float* v, int n_chunks, int64_t N,
-                                const float* dt, const int32_t* step, int m, float eps, float* f,
-                                float* l1, uint8_t* mask, cudaStream_t s) {
-  if (n_chunks < 1 || n_chunks > kGateNoAllocMaxChunks) return cudaErrorInvalidValue;
+cudaError_t gate_noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -406,7 +403,17 @@ cudaError_t launch_gate_noalloc(float* x, const float* v, int n_chunks, int64_t 
     if (e != cudaSuccess) return e;
     g_gate_scratch_addr[dev] = p;
   }
-  void* ws = g_gate_scratch_addr[dev];
+  *out = g_gate_scratch_addr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_gate_noalloc(float* x, const float* v, int n_chunks, int64_t N,
+                                const float* dt, const int32_t* step, int m, float eps, float* f,
+                                float* l1, uint8_t* mask, cudaStream_t s) {
+  if (n_chunks < 1 || n_chunks > kGateNoAllocMaxChunks) return cudaErrorInvalidValue;
+  void* ws = nullptr;
+  cudaError_t e = gate_noalloc_scratch(&ws);
+  if (e != cudaSuccess) return e;
   // The completion counters and the error word must start at zero; the array
   // keeps whatever the previous call left, so clear them on the caller's
   // stream first.

@@ -47,7 +47,7 @@ typedef enum {
   FC_ERR_UNSUPPORTED = 2, /* a valid request this build does not implement         */
   FC_ERR_WORKSPACE = 3,   /* ws is null or smaller than the *_workspace_size()     */
   FC_ERR_CUDA = 4,        /* a CUDA call failed; see fc_last_error()               */
-  FC_ERR_TIMEOUT = 5      /* reserved: a bounded device-side wait gave up          */
+  FC_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up (fc_check_workspace) */
 } fc_status;
 
 typedef enum { FC_F32 = 0, FC_BF16 = 1 } fc_dtype;
@@ -57,6 +57,32 @@ const char* fc_last_error(void);
 
 /* Library version, as major*10000 + minor*100 + patch. */
 int fc_version(void);
+
+/*
+ * Failure detection for the calls whose kernels wait on the device (the gate's
+ * streaming path, the importance, the cache commit): every such wait is
+ * bounded, and a wait that gives up sets a 32-bit error word in the call's
+ * workspace and lets the kernel return instead of hanging.  The calls are
+ * asynchronous, so the word is read here, after the work is done.
+ *
+ *   kind      which call's workspace ws is (the word's place differs)
+ *   ws        the workspace passed to that call (ignored for FC_WS_GATE_NOALLOC,
+ *             whose scratch is the library's own on the current device)
+ *   n_chunks  the call's n_chunks (gate kinds only)
+ *   clear     nonzero: reset a set word to zero after reading it
+ * Synchronises `stream`, then returns FC_OK if the word is zero and
+ * FC_ERR_TIMEOUT if it is set (the outputs of the calls made since it was last
+ * zero are not valid).  Bad arguments -> FC_ERR_INVALID_ARG; a failed read ->
+ * FC_ERR_CUDA.  The pages have no counterpart: this is the library's own.
+ */
+typedef enum {
+  FC_WS_GATE = 0,          /* fc_chunk_l1_gate / fc_history_l1_gate workspace  */
+  FC_WS_GATE_NOALLOC = 1,  /* fc_chunk_l1_gate_noalloc's static scratch       */
+  FC_WS_IMPORTANCE = 2,    /* fc_kv_importance workspace                      */
+  FC_WS_CACHE = 3          /* fc_kv_cache_commit workspace                    */
+} fc_ws_kind;
+fc_status fc_check_workspace(fc_ws_kind kind, const void* ws, int n_chunks, int clear,
+                             void* stream);
 
 /* Kernel launches (memsets included) that the last compute call made on this
  * host thread enqueued; 0 after an error.  For accounting in benchmarks. */

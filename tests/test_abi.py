@@ -181,3 +181,13 @@ def test_cache_commit_validates_and_keeps_fitting_chunks_on_the_host():
     assert (n_next.value, comp.value) == (-1, -1)
     assert lib.fc_kv_cache_workspace_size(fc.FC_BF16, 2, 8, 96, 32, 64) > 0
     assert lib.fc_kv_cache_workspace_size(fc.FC_BF16, 2, 8, 96, 32, 96) == 0
+
+
+def test_check_workspace_validates_on_the_host():
+    lib = fc.library()
+    assert lib.fc_check_workspace(9, NULL, 1, 0, NULL) == 1  # unknown kind
+    assert lib.fc_check_workspace(fc.FC_WS_GATE, NULL, 0, 0, NULL) == 1  # n_chunks < 1
+    assert lib.fc_check_workspace(fc.FC_WS_GATE, NULL, 4, 0, NULL) == 1
+    assert lib.fc_last_error() == b"ws is NULL"
+    assert lib.fc_check_workspace(fc.FC_WS_IMPORTANCE, NULL, 0, 0, NULL) == 1
+    assert lib.fc_check_workspace(fc.FC_WS_GATE_NOALLOC, NULL, 33, 0, NULL) == 1  # > 32 chunks
