@@ -39,6 +39,14 @@ sys.path.insert(0, ROOT)
 METRIC = "clean KV tokens scored+selected/s per head; L1-gate GB/s; % of roofline"
 UNIT = "tokens/s/head"
 FLUSH_BYTES = 256 << 20  # > 126 MB L2
+# Exponentials per SM clock of a B200 probe mixing the special-function unit
+# and an FMA-pipe polynomial 5:3, with nothing else running: the exp ceiling
+# the importance epilogue is measured against.
+EXP_PROBE_PER_CLK = 20.6
+
+
+def _sms(dev):
+    return torch.cuda.get_device_properties(dev).multi_processor_count
 
 
 def flush_l2(buf, sink):
@@ -263,12 +271,13 @@ class Step:
              "compact": ("score1", "end")}
     EVENTS = ("start", "gate0", "gate1", "red1", "imp0", "imp1", "join", "score1", "end")
 
-    def run(self, stream, ev=None, side=None):
+    def run(self, stream, ev=None, side=None, side_after=(), compact_after=()):
         """Enqueue one step; returns the number of kernel launches the library
         enqueued.  The gate and the redundancy depend on nothing else in the
         step, so with a ``side`` stream they run there, beside the importance
         on ``stream``, and the score waits for both.  ``ev`` maps the names in
-        EVENTS to timing events."""
+        EVENTS to timing events.  ``side_after`` / ``compact_after``: events the
+        gate / the compaction must wait for (inputs still being copied in)."""
         fc, d, o, w = self.fc, self.d, self.out, self.ws
         rec = (lambda k, st: ev[k].record(st)) if ev else (lambda k, st: None)
         s2 = side if side is not None else stream
@@ -277,6 +286,8 @@ class Step:
         if side is not None:
             self.fork.record(stream)
             side.wait_event(self.fork)
+        for e in side_after:
+            s2.wait_event(e)
         rec("gate0", s2)
         if self.n_c:
             fc.fc_chunk_l1_gate(d["x"], d["vel"], d["dt"], d["step"], self.gc.m, self.eps,
@@ -298,6 +309,8 @@ class Step:
                             w["topb"], stream=stream)
         n += fc.fc_last_launches()
         rec("score1", stream)
+        for e in compact_after:
+            stream.wait_event(e)
         fc.fc_kv_compact(d["k"], d["v"], o["idx"], o["ko"], o["vo"], stream=stream)
         n += fc.fc_last_launches()
         rec("end", stream)
@@ -445,6 +458,7 @@ def native(a, rank, world, local_rank):
     hbm, tf_burst, tf_sus, src = _peaks()
     exec_flops = 4.0 * H * Lq * Lk * d  # two passes of Q K^T
     imp_tf = exec_flops / (ms_call["importance"] * 1e-3) / 1e12
+    gexp = 2.0 * H * Lq * Lk / (ms_call["importance"] * 1e-3) / 1e9
     gate_gbs = (_bytes_gate(gate_cfg) * step.n_c / gate_cfg.n_chunks / (ms_alone["gate"] * 1e-3)
                 / 1e9) if step.n_c else None
     elem = 2 if kv_cfg.dtype == "bf16" else 4
@@ -488,9 +502,12 @@ def native(a, rank, world, local_rank):
                    "stream beside the importance (they depend on nothing else in the step)") +
                   f"; eager (host-launched) step for reference: {ms_eager:.3f} ms",
         "importance": {"TFLOP/s executed": imp_tf, "TFLOP/s algorithmic": imp_tf / 2,
-                       "Gexp/s": 2.0 * H * Lq * Lk / (ms_call["importance"] * 1e-3) / 1e9,
+                       "Gexp/s": gexp,
+                       "frac_of_exp_probe": gexp * 1e9 / (EXP_PROBE_PER_CLK * _sms(dev) *
+                                                         (ck.get("sm_mhz") or 1965) * 1e6),
                        "note": "both passes recompute Q K^T (executed = 2 x algorithmic "
-                               "flops); 2 exponentials per score"},
+                               "flops); 2 exponentials per score; frac_of_exp_probe: against "
+                               f"{EXP_PROBE_PER_CLK} exps/clock/SM at the sampled SM clock"},
         "redundancy": {"GB/s": red_gbs, "frac_hbm": red_gbs / hbm},
         "score_topb": {"GB/s": topb_gbs},
         "compact": {"GB/s": comp_gbs, "frac_hbm": comp_gbs / hbm},
@@ -634,15 +651,38 @@ def _e2e(step, stream, side, flush, sink, a, dev):
         host_out["f"] = torch.empty_like(step.host["f"]).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_in.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out.values())
+    # With a side stream the copies are ordered for overlap: Q and K first (the
+    # importance and the redundancy need them), then the gate's inputs and V on
+    # a copy stream while the importance runs; the gate waits for its inputs,
+    # the compaction for V.  The PCIe link carries one copy after another.
+    first = [n for n in ("q", "k") if n in host_in]
+    later = [n for n in host_in if n not in first and n != "v"] + ["v"]
+    cp = torch.cuda.Stream(device=dev) if side is not None else None
     times = []
     with torch.cuda.stream(stream):
         for i in range(a.warmup + a.steps):
             flush_l2(flush, sink)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
-            for n, t in host_in.items():
-                step.d[n].copy_(t, non_blocking=True)
-            step.run(stream, side=side)
+            if cp is None:
+                for n, t in host_in.items():
+                    step.d[n].copy_(t, non_blocking=True)
+                step.run(stream)
+            else:
+                for n in first:
+                    step.d[n].copy_(host_in[n], non_blocking=True)
+                qk = torch.cuda.Event()
+                qk.record(stream)
+                cp.wait_event(qk)
+                with torch.cuda.stream(cp):
+                    for n in later[:-1]:
+                        step.d[n].copy_(host_in[n], non_blocking=True)
+                    gate_in = torch.cuda.Event()
+                    gate_in.record(cp)
+                    step.d["v"].copy_(host_in["v"], non_blocking=True)
+                    v_in = torch.cuda.Event()
+                    v_in.record(cp)
+                step.run(stream, side=side, side_after=(gate_in,), compact_after=(v_in,))
             for n in res:
                 host_out[n].copy_(step.d["f"] if n == "f" else step.out[n], non_blocking=True)
             e1.record(stream)
