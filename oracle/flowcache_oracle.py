@@ -29,7 +29,7 @@ kernel's precision, so that both sides take every integer decision the same
 way).  Matrix products and sorts are library calls (numpy); nothing is blocked
 or fused beyond processing independent rows of a matrix a group at a time.
 
-Readings of points the pages leave open (each also listed in the design doc):
+Readings of points the pages leave open:
 the mask is the decision for the chunk's next forward; "first m steps" counts
 per chunk; the comparison with eps is strict; ||X_t||_1 = 0 gives L1 = +inf
 (or 0 when the update is also zero); a step counter < 0 marks an inactive

@@ -124,8 +124,9 @@ def test_gate_theorem1_monotone_on_flow_matching_toy(seed):
     """Theorem 1: at the exact flow-matching velocity with sigma(t) = (t/T)^p,
     L1_rel rises monotonically along the trajectory.  Toy: single-point data
     x0 (std 0.1), x_s = s*x0 + (1-s)*noise, exact velocity x0 - noise, Euler
-    steps dt = sigma(t+1) - sigma(t), p = 2, T = 30 (the regime in which the
-    theorem's unstated assumptions hold is recorded in the design doc)."""
+    steps dt = sigma(t+1) - sigma(t), p = 2, T = 30.  The pages do not print the
+    theorem's assumptions; the rise is regime dependent (a large x0, or p <= 1,
+    breaks it), and this is a regime where it holds."""
     rng = np.random.default_rng(100 + seed)
     N, T, p = 16384, 30, 2.0
     x0 = rng.standard_normal(N) * 0.1
