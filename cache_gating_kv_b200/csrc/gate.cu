@@ -9,16 +9,18 @@
 //
 // Design (B200): the pass moves 12 bytes per element (read X, read v, write
 // X), so it is bound by HBM.  The grid is n_chunks x blocks_per_chunk with the
-// total sized to fill all SMs; every thread streams 16-byte vectors with
-// read-once cache hints, unrolled so that each thread keeps eight loads in
-// flight.  Partial sums are float64 (exact enough that the float32 L1_rel is
+// total sized to fill all SMs (four resident blocks per SM); every thread
+// streams 16-byte vectors with read-once cache hints, unrolled so that each
+// thread keeps eight loads in flight, and the first of them go out before the
+// chunk's step counter and dt are read.  (Staging the stream through shared
+// memory with 1-D TMA bulk copies, one CTA per SM, measured 14% slower at 4
+// chunks and 6% slower at 16 on B200.)  Partial sums are float64 (exact enough that the float32 L1_rel is
 // practically the correctly rounded quotient).  Each block stores its partial
 // pair; the last block of a chunk to finish (an integer completion counter,
 // no spinning, no float atomics) sums the partials in a fixed order and runs
 // the recurrence, so the result is deterministic and one launch does it all.
 #include "fc_common.cuh"
 #include "fc_kernels.h"
-#include "tc_ptx.cuh"
 
 namespace fc {
 
@@ -75,15 +77,6 @@ __global__ void __launch_bounds__(kGateThreads)
   const int c = blockIdx.y;
   const int b = blockIdx.x;
   const int tid = threadIdx.x;
-  const int st = step[c];
-  if (st < 0) {  // inactive chunk: nothing touched
-    if (b == 0 && tid == 0) {
-      l1[c] = 0.0f;
-      mask[c] = 0;
-    }
-    return;
-  }
-  const float h = kHist ? 0.0f : dt[c];
   const int64_t off = (int64_t)c * N;
   float* xc = x + off;
   const float* vc = v + off;
@@ -100,18 +93,33 @@ __global__ void __launch_bounds__(kGateThreads)
   const int64_t hi = min(nvec, lo + per);
   float4* x4 = reinterpret_cast<float4*>(xc + head);
   const float4* v4 = reinterpret_cast<const float4*>(vc + head);
+  constexpr int64_t kStride = (int64_t)kGateThreads * kGateUnroll;
+
+  // The first loads go out before the chunk's step and dt are read, so the
+  // stream does not wait behind those two dependent loads; nothing is written
+  // before the step is known.
+  float4 xa[kGateUnroll], va[kGateUnroll];
+  int64_t base = lo + tid;
+#pragma unroll
+  for (int u = 0; u < kGateUnroll; ++u) {
+    const int64_t i = base + (int64_t)u * kGateThreads;
+    if (i < hi) {
+      xa[u] = __ldcs(x4 + i);
+      va[u] = __ldcs(v4 + i);
+    }
+  }
+  const int st = step[c];
+  const float h = kHist ? 0.0f : dt[c];
+  if (st < 0) {  // inactive chunk: nothing touched
+    if (b == 0 && tid == 0) {
+      l1[c] = 0.0f;
+      mask[c] = 0;
+    }
+    return;
+  }
 
   double num = 0.0, den = 0.0;
-  for (int64_t base = lo + tid; base < hi; base += (int64_t)kGateThreads * kGateUnroll) {
-    float4 xa[kGateUnroll], va[kGateUnroll];
-#pragma unroll
-    for (int u = 0; u < kGateUnroll; ++u) {
-      const int64_t i = base + (int64_t)u * kGateThreads;
-      if (i < hi) {
-        xa[u] = __ldcs(x4 + i);
-        va[u] = __ldcs(v4 + i);
-      }
-    }
+  for (; base < hi; base += kStride) {
 #pragma unroll
     for (int u = 0; u < kGateUnroll; ++u) {
       const int64_t i = base + (int64_t)u * kGateThreads;
@@ -121,6 +129,14 @@ __global__ void __launch_bounds__(kGateThreads)
         gate_elem<kHist>(xa[u].z, va[u].z, h, num, den);
         gate_elem<kHist>(xa[u].w, va[u].w, h, num, den);
         __stcs(x4 + i, xa[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kGateUnroll; ++u) {
+      const int64_t i = base + kStride + (int64_t)u * kGateThreads;
+      if (i < hi) {
+        xa[u] = __ldcs(x4 + i);
+        va[u] = __ldcs(v4 + i);
       }
     }
   }
@@ -181,140 +197,11 @@ __global__ void __launch_bounds__(kGateThreads)
     }
   }
 }
-// ---------------------------------------------------------------------------
-// Streaming variant for chunks of whole 16-byte vectors (N % 4 == 0): one CTA
-// per SM-share of a chunk pulls its slice of X and v through a ring of
-// shared-memory stages with 1-D TMA bulk copies (thread 0 keeps every stage
-// in flight), the 256 threads compute from shared memory and write X back
-// with 16-byte stores.  The partial sums are published before the last
-// stores drain, so the finalising block is not held up by them.
-// ---------------------------------------------------------------------------
-constexpr int kSegFloats = 4096;  // one stage: 16 KB of X + 16 KB of v
-constexpr int kSegStages = 6;     // 192 KB of loads in flight per CTA
-constexpr int kTmaThreads = 256;
-
-struct GateStage {
-  float x[kSegFloats];
-  float v[kSegFloats];
-};
-
-template <bool kHist>
-__global__ void __launch_bounds__(kTmaThreads, 1)
-    gate_tma_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t N,
-                    const float* __restrict__ dt, const int32_t* __restrict__ step, int m,
-                    float eps, float* __restrict__ f, float* __restrict__ l1,
-                    uint8_t* __restrict__ mask, unsigned* __restrict__ counters,
-                    double2* __restrict__ partials, int bpc, int* __restrict__ err) {
-  extern __shared__ __align__(128) unsigned char gsm[];
-  GateStage* stages = reinterpret_cast<GateStage*>(gsm);
-  uint64_t* full = reinterpret_cast<uint64_t*>(gsm + kSegStages * sizeof(GateStage));
-  __shared__ double s_num[kTmaThreads / 32], s_den[kTmaThreads / 32];
-  __shared__ int s_last;
-
-  const int c = blockIdx.y, b = blockIdx.x, tid = threadIdx.x;
-  const int warp = tid >> 5, lane = tid & 31;
-  const int st = step[c];
-  if (st < 0) {  // inactive chunk: nothing touched
-    if (b == 0 && tid == 0) {
-      l1[c] = 0.0f;
-      mask[c] = 0;
-    }
-    return;
-  }
-  const float h = kHist ? 0.0f : dt[c];
-  // This block's slice of the chunk, in whole vectors.
-  const int64_t nvec = N >> 2;
-  const int64_t per = ceil_div(nvec, bpc);
-  const int64_t v_lo = min(nvec, per * b), v_hi = min(nvec, v_lo + per);
-  float* xs = x + (size_t)c * N + v_lo * 4;
-  const float* vs = v + (size_t)c * N + v_lo * 4;
-  const int64_t n = (v_hi - v_lo) * 4;  // floats in the slice
-  const int nseg = (int)ceil_div(n, kSegFloats);
-
-  if (tid == 0) {
-    for (int sidx = 0; sidx < kSegStages; ++sidx) tc::mbar_init(&full[sidx], 1);
-    tc::fence_barrier_init();
-  }
-  __syncthreads();
-  auto issue = [&](int seg) {
-    const int sidx = seg % kSegStages;
-    const int64_t off = (int64_t)seg * kSegFloats;
-    const uint32_t bytes = (uint32_t)(min((int64_t)kSegFloats, n - off) * 4);
-    tc::mbar_expect_tx(&full[sidx], 2 * bytes);
-    tc::bulk_load(stages[sidx].x, xs + off, bytes, &full[sidx]);
-    tc::bulk_load(stages[sidx].v, vs + off, bytes, &full[sidx]);
-  };
-  if (tid == 0)
-    for (int seg = 0; seg < kSegStages && seg < nseg; ++seg) issue(seg);
-
-  double num = 0.0, den = 0.0;
-  bool ok = true;
-  for (int seg = 0; seg < nseg; ++seg) {
-    const int sidx = seg % kSegStages;
-    const bool landed = tc::mbar_wait(&full[sidx], (seg / kSegStages) & 1);
-    if (!__syncthreads_and(landed)) {  // the whole block leaves together on a timeout
-      ok = false;
-      break;
-    }
-    const int64_t off = (int64_t)seg * kSegFloats;
-    const int cnt4 = (int)(min((int64_t)kSegFloats, n - off) >> 2);
-    const float4* sx = reinterpret_cast<const float4*>(stages[sidx].x);
-    const float4* sv = reinterpret_cast<const float4*>(stages[sidx].v);
-    float4* gx = reinterpret_cast<float4*>(xs + off);
-    for (int i = tid; i < cnt4; i += kTmaThreads) {
-      float4 xa = sx[i];
-      gate_elem<kHist>(xa.x, sv[i].x, h, num, den);
-      gate_elem<kHist>(xa.y, sv[i].y, h, num, den);
-      gate_elem<kHist>(xa.z, sv[i].z, h, num, den);
-      gate_elem<kHist>(xa.w, sv[i].w, h, num, den);
-      __stcs(gx + i, xa);
-    }
-    __syncthreads();  // stage sidx fully consumed
-    if (tid == 0 && seg + kSegStages < nseg) issue(seg + kSegStages);
-  }
-
-  num = warp_sum(num);
-  den = warp_sum(den);
-  if (lane == 0) {
-    s_num[warp] = num;
-    s_den[warp] = den;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    if (!ok) atomicExch(err, 1);
-    double a = 0.0, d = 0.0;
-#pragma unroll
-    for (int w = 0; w < kTmaThreads / 32; ++w) {
-      a += s_num[w];
-      d += s_den[w];
-    }
-    partials[(size_t)c * kGateMaxBlocksPerChunk + b] = make_double2(a, d);
-    __threadfence();
-    const unsigned prev = atomicAdd(&counters[c], 1u);
-    s_last = (prev == (unsigned)(bpc - 1));
-  }
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  if (warp == 0) {
-    double a = 0.0, d = 0.0;
-    for (int i = lane; i < bpc; i += 32) {
-      const double2 p = __ldcg(&partials[(size_t)c * kGateMaxBlocksPerChunk + i]);
-      a += p.x;
-      d += p.y;
-    }
-    a = warp_sum(a);
-    d = warp_sum(d);
-    if (lane == 0) {
-      gate_finalize<kHist>(c, st, m, eps, a, d, f, l1, mask);
-      counters[c] = 0u;
-    }
-  }
-}
 }  // namespace
 
-// Workspace: completion counters [n_chunks], an error word, then the
-// per-block partial sums [n_chunks][kGateMaxBlocksPerChunk].
+// Workspace: completion counters [n_chunks], an error word (the gate has no
+// device-side waits, so it stays zero), then the per-block partial sums
+// [n_chunks][kGateMaxBlocksPerChunk].
 static size_t counters_bytes(int n_chunks) {
   return align_up((size_t)(n_chunks + 1) * sizeof(unsigned), 256);
 }
@@ -327,26 +214,8 @@ cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t N, const
                         const int32_t* step, int m, float eps, float* f, float* l1,
                         uint8_t* mask, void* ws, cudaStream_t s, bool history) {
   unsigned* counters = static_cast<unsigned*>(ws);
-  int* err = reinterpret_cast<int*>(counters + n_chunks);
   double2* partials =
       reinterpret_cast<double2*>(static_cast<char*>(ws) + counters_bytes(n_chunks));
-  if (N >= 4 * 1024 && N % 4 == 0) {
-    // Streaming path: at most one CTA per SM over all chunks (one wave).
-    int64_t bpc = (int64_t)sm_count() / n_chunks;
-    const int64_t useful = ceil_div(N / 4, 1024);  // >= 4 KB per block
-    if (bpc > useful) bpc = useful;
-    if (bpc < 1) bpc = 1;
-    if (bpc > kGateMaxBlocksPerChunk) bpc = kGateMaxBlocksPerChunk;
-    const size_t smem = (size_t)kSegStages * sizeof(GateStage) + kSegStages * sizeof(uint64_t);
-    auto kern = history ? gate_tma_kernel<true> : gate_tma_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
-    if (e != cudaSuccess) return e;
-    kern<<<dim3((unsigned)bpc, (unsigned)n_chunks), kTmaThreads, smem, s>>>(
-        x, v, N, dt, step, m, eps, f, l1, mask, counters, partials, (int)bpc, err);
-    add_launches(1);
-    return cudaGetLastError();
-  }
   // Four resident 256-thread blocks per SM over the whole grid.
   const int64_t target = (int64_t)sm_count() * 4;
   int64_t bpc = ceil_div(target, n_chunks);

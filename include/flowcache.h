@@ -59,11 +59,12 @@ const char* fc_last_error(void);
 int fc_version(void);
 
 /*
- * Failure detection for the calls whose kernels wait on the device (the gate's
- * streaming path, the importance, the cache commit): every such wait is
- * bounded, and a wait that gives up sets a 32-bit error word in the call's
- * workspace and lets the kernel return instead of hanging.  The calls are
- * asynchronous, so the word is read here, after the work is done.
+ * Failure detection for the calls whose kernels wait on the device (the
+ * importance and the cache commit; the gate's kernel has no device-side waits
+ * and leaves its word zero, but its workspace keeps the word): every such
+ * wait is bounded, and a wait that gives up sets a 32-bit error word in the
+ * call's workspace and lets the kernel return instead of hanging.  The calls
+ * are asynchronous, so the word is read here, after the work is done.
  *
  *   kind      which call's workspace ws is (the word's place differs)
  *   ws        the workspace passed to that call (ignored for FC_WS_GATE_NOALLOC,
@@ -128,9 +129,8 @@ size_t fc_gate_workspace_size(int n_chunks, int64_t n_per_chunk);
  *              bytes (completion counters and an error word) must be zero
  *              before the first call (e.g. cudaMemsetAsync once); every call
  *              leaves the counters zero again.  The error word (the 32-bit
- *              word after the n_chunks counters) becomes nonzero if a bounded
- *              device-side wait of the streaming path gave up; the call never
- *              clears it.
+ *              word after the n_chunks counters) is reserved: this kernel
+ *              has no device-side waits and never sets it.
  * x and v may be NULL when n_per_chunk == 0 (then L1_rel = 0 for every
  * active chunk).
  * Errors: n_chunks < 1, n_per_chunk < 0, m < 0, null/host/misaligned
