@@ -464,7 +464,7 @@ def native(a, rank, world, local_rank):
     elem = 2 if kv_cfg.dtype == "bf16" else 4
     red_gbs = H * Lk * d * elem / (ms_alone["redundancy"] * 1e-3) / 1e9
     comp_gbs = 2 * 2 * H * kv_cfg.B * d * elem / (ms_alone["compact"] * 1e-3) / 1e9
-    topb_gbs = H * Lk * 12 / (ms_alone["score_topb"] * 1e-3) / 1e9
+    topb_gbs = (H * Lk * 8 + H * kv_cfg.B * 4) / (ms_alone["score_topb"] * 1e-3) / 1e9
     launches = launches_per_step * a.steps
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
@@ -509,7 +509,8 @@ def native(a, rank, world, local_rank):
                                "flops); 2 exponentials per score; frac_of_exp_probe: against "
                                f"{EXP_PROBE_PER_CLK} exps/clock/SM at the sampled SM clock"},
         "redundancy": {"GB/s": red_gbs, "frac_hbm": red_gbs / hbm},
-        "score_topb": {"GB/s": topb_gbs},
+        "score_topb": {"GB/s": topb_gbs, "frac_hbm": topb_gbs / hbm,
+                       "bytes": "8 B read per token (imp, red) + 4 B written per kept index"},
         "compact": {"GB/s": comp_gbs, "frac_hbm": comp_gbs / hbm},
         "gpu_launches": launches,
         "clocks": ck,
