@@ -204,8 +204,9 @@ __global__ void __launch_bounds__(kSelThreads)
 // digit), and the final ordered compaction offsets each CTA by the kept
 // counts of the CTAs before it.  Cluster barriers are hardware barriers.
 // ---------------------------------------------------------------------------
-constexpr int kCsThreads = 256;
+constexpr int kCsThreads = 512;  // 256 measured 8 % (L_k 16384) to 27 % (131072) slower
 constexpr int kCsWarps = kCsThreads / 32;
+static_assert(kCsThreads >= 256, "one thread per histogram bin");
 constexpr int kCsMaxSlice = 12288;  // keys per CTA held in shared memory
 
 __global__ void __launch_bounds__(kCsThreads)
@@ -276,14 +277,14 @@ __global__ void __launch_bounds__(kCsThreads)
       }
     }
     __syncthreads();
-    {
+    if (tid < 256) {  // one thread per bin
       unsigned t = 0u;
 #pragma unroll
       for (int w = 0; w < kCsWarps; ++w) t += whist[w][tid];
-      hist[pass & 1][tid] = t;  // kCsThreads == 256 bins
+      hist[pass & 1][tid] = t;
     }
     cluster.sync();
-    {
+    if (tid < 256) {
       unsigned t = 0u;
       for (int q = 0; q < nrank; ++q) t += *cluster.map_shared_rank(&hist[pass & 1][tid], q);
       s_total[tid] = t;
