@@ -23,7 +23,7 @@
 // holds two 16-byte vectors of a row (16 bf16 or 8 fp32 elements), so a row's
 // reductions take log2(d*elem/32) shuffles; the per-row scalars use the
 // special-function unit (rsqrt, ex2: ~2^-22 relative error); every lane keeps
-// four rows' loads in flight.
+// two or four rows' loads in flight.
 #include <cooperative_groups.h>
 
 #include "fc_common.cuh"
@@ -36,7 +36,6 @@ namespace fc {
 namespace {
 constexpr int kRedThreads = 256;
 constexpr int kRedWarps = kRedThreads / 32;
-constexpr int kRedUnroll = 2;  // rows in flight per lane (two 16-byte loads each)
 
 // Each lane holds two 16-byte vectors (32 contiguous bytes) of a row.
 template <typename T, int D>
@@ -67,12 +66,12 @@ __device__ __forceinline__ float row_sum(float v) {
   return v;
 }
 
-template <typename T, int D>
+template <typename T, int D, int U>
 __device__ __forceinline__ void load_rows(const T* kh, int r0, int hi, int sub, int cl,
-                                          uint4 (&u)[kRedUnroll][2]) {
+                                          uint4 (&u)[U][2]) {
   using L = RowLayout<T, D>;
 #pragma unroll
-  for (int i = 0; i < kRedUnroll; ++i) {
+  for (int i = 0; i < U; ++i) {
     const int r = r0 + i * L::RPW + sub;
     const T* p = kh + (size_t)r * D + cl * L::EPL;
     u[i][0] = r < hi ? ld_nc_v4(p) : make_uint4(0u, 0u, 0u, 0u);
@@ -86,7 +85,8 @@ __device__ __forceinline__ void unpack(const uint4 (&u)[2], float* e) {
   Vec16<T>::to_float(u[1], e + Vec16<T>::N);
 }
 
-template <typename T, int D>
+// U: rows in flight per lane (two 16-byte loads each).
+template <typename T, int D, int U>
 __global__ void __launch_bounds__(kRedThreads)
     red_cluster_kernel(const T* __restrict__ k, int Lk, int h0, float* __restrict__ red) {
   using L = RowLayout<T, D>;
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(kRedThreads)
   const int per = (int)ceil_div(Lk, nrank);
   const int lo = min(Lk, rank * per), hi = min(Lk, lo + per);
   const T* kh = k + (size_t)h * Lk * D;
-  constexpr int kRowsPerIter = kRedWarps * L::RPW * kRedUnroll;
+  constexpr int kRowsPerIter = kRedWarps * L::RPW * U;
 
   __shared__ float s_acc[kRedWarps][D];
   __shared__ float s_part[D];  // this CTA's sum of khat (read by the whole cluster)
@@ -112,11 +112,11 @@ __global__ void __launch_bounds__(kRedThreads)
   float acc[L::EPL];
 #pragma unroll
   for (int i = 0; i < L::EPL; ++i) acc[i] = 0.0f;
-  for (int r0 = lo + warp * L::RPW * kRedUnroll; r0 < hi; r0 += kRowsPerIter) {
-    uint4 raw[kRedUnroll][2];
-    load_rows<T, D>(kh, r0, hi, sub, cl, raw);
+  for (int r0 = lo + warp * L::RPW * U; r0 < hi; r0 += kRowsPerIter) {
+    uint4 raw[U][2];
+    load_rows<T, D, U>(kh, r0, hi, sub, cl, raw);
 #pragma unroll
-    for (int u = 0; u < kRedUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       float e[L::EPL];
       unpack<T, D>(raw[u], e);
       float n2 = 0.0f;
@@ -162,11 +162,11 @@ __global__ void __launch_bounds__(kRedThreads)
   // they are still in L2.
   const int n_iter = (int)ceil_div(hi - lo, kRowsPerIter);
   for (int it = n_iter - 1; it >= 0; --it) {
-    const int r0 = lo + it * kRowsPerIter + warp * L::RPW * kRedUnroll;
-    uint4 raw[kRedUnroll][2];
-    load_rows<T, D>(kh, r0, hi, sub, cl, raw);
+    const int r0 = lo + it * kRowsPerIter + warp * L::RPW * U;
+    uint4 raw[U][2];
+    load_rows<T, D, U>(kh, r0, hi, sub, cl, raw);
 #pragma unroll
-    for (int u = 0; u < kRedUnroll; ++u) {
+    for (int u = 0; u < U; ++u) {
       float e[L::EPL];
       unpack<T, D>(raw[u], e);
       float n2 = 0.0f, dot = 0.0f;
@@ -214,7 +214,9 @@ template <typename T, int D>
 cudaError_t run(const T* k, int H, int Lk, float* red, cudaStream_t s) {
   // 16 CTAs per head when the slices stay long enough, else the portable 8.
   const int csize = (Lk >= 16 * 64) ? 16 : 8;
-  auto kern = red_cluster_kernel<T, D>;
+  // Long heads keep four rows per lane in flight (two measured 17 % slower at
+  // L_k = 131072); short ones two (four measured 17 % slower at 16384).
+  auto kern = Lk >= 65536 ? red_cluster_kernel<T, D, 4> : red_cluster_kernel<T, D, 2>;
   if (csize > 8) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     if (e != cudaSuccess) return e;
