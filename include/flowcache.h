@@ -14,8 +14,10 @@
  * Conventions shared by every call
  *   - Every tensor pointer is a DEVICE pointer (cudaMalloc / torch CUDA
  *     memory / managed memory) owned by the caller.  The library allocates
- *     nothing and keeps no state between calls.  Host pointers are rejected
- *     with FC_ERR_INVALID_ARG before anything is launched.
+ *     nothing and keeps no state between calls, except the static scratch
+ *     array that fc_chunk_l1_gate_noalloc uses instead of a workspace.  Host
+ *     pointers are rejected with FC_ERR_INVALID_ARG before anything is
+ *     launched.
  *   - Tensors are dense, row-major, with the stated layout, and their base
  *     address is 16-byte aligned.  "[H][L][d]" means head-major.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls
@@ -252,7 +254,7 @@ size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d
  *   ws     fc_importance_workspace_size() bytes: bytes 0..3 are an error
  *          word that the tensor-core path sets to nonzero if one of its
  *          bounded device-side waits gave up (the call never clears it; zero
- *          it once, read it after synchronizing); the per-query log-sum-exp
+ *          it once; read it with fc_check_workspace); the per-query log-sum-exp
  *          follows from byte 256
  * Errors: H, Lq, Lk < 1 or d not in {64, 128} -> FC_ERR_INVALID_ARG /
  * FC_ERR_UNSUPPORTED; bad pointers -> FC_ERR_INVALID_ARG; small ws ->
