@@ -4,6 +4,8 @@
 #include <cstdio>
 #include <cstring>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/flowcache.h"
 #include "../../include/flowcache_selftest.h"
 #include "fc_common.cuh"
@@ -40,6 +42,15 @@ fc_status fail(fc_status st, const char* fmt, ...) {
   va_end(ap);
   return st;
 }
+
+// An NVTX range around each compute call, named after it, so that a profiler
+// timeline shows the library's calls (no cost without a profiler attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 fc_status ok() {
   g_err[0] = '\0';
@@ -133,6 +144,7 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
                            const float* dt, const int32_t* step, int32_t m, float eps, float* f,
                            float* l1_rel, uint8_t* recompute, void* ws, size_t ws_bytes,
                            void* stream) {
+  NvtxRange _range("fc_chunk_l1_gate");
   fc::g_launches = 0;
   if (n_chunks < 1 || n_chunks > 65535)
     return fail(FC_ERR_INVALID_ARG, "n_chunks must be in [1, 65535] (got %d)", n_chunks);
@@ -159,6 +171,7 @@ fc_status fc_history_l1_gate(float* h_old, const float* h_new, int n_segments,
                              int64_t n_per_segment, const int32_t* step, int32_t m, float delta,
                              float* f, float* d_rel, uint8_t* refresh, void* ws, size_t ws_bytes,
                              void* stream) {
+  NvtxRange _range("fc_history_l1_gate");
   fc::g_launches = 0;
   if (n_segments < 1 || n_segments > 65535)
     return fail(FC_ERR_INVALID_ARG, "n_segments must be in [1, 65535] (got %d)", n_segments);
@@ -183,6 +196,7 @@ fc_status fc_history_l1_gate(float* h_old, const float* h_new, int n_segments,
 fc_status fc_chunk_l1_gate_noalloc(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
                                    const float* dt, const int32_t* step, int32_t m, float eps,
                                    float* f, float* l1_rel, uint8_t* recompute, void* stream) {
+  NvtxRange _range("fc_chunk_l1_gate_noalloc");
   fc::g_launches = 0;
   const int max_chunks = fc::gate_noalloc_max_chunks();
   if (n_chunks < 1 || n_chunks > max_chunks)
@@ -209,6 +223,7 @@ fc_status fc_chunk_l1_gate_noalloc(float* x, const float* v, int n_chunks, int64
 fc_status fc_gather_recompute(const float* x, const uint8_t* recompute, int n_chunks,
                               int64_t n_per_chunk, float* dense, int32_t* ids, int32_t* count,
                               void* stream) {
+  NvtxRange _range("fc_gather_recompute");
   fc::g_launches = 0;
   if (n_chunks < 1 || n_chunks > 65535)
     return fail(FC_ERR_INVALID_ARG, "n_chunks must be in [1, 65535] (got %d)", n_chunks);
@@ -227,6 +242,7 @@ fc_status fc_gather_recompute(const float* x, const uint8_t* recompute, int n_ch
 
 fc_status fc_scatter_velocity(const float* v_dense, const int32_t* ids, const int32_t* count,
                               int n_chunks, int64_t n_per_chunk, float* v_cache, void* stream) {
+  NvtxRange _range("fc_scatter_velocity");
   fc::g_launches = 0;
   if (n_chunks < 1 || n_chunks > 65535)
     return fail(FC_ERR_INVALID_ARG, "n_chunks must be in [1, 65535] (got %d)", n_chunks);
@@ -299,6 +315,7 @@ size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d
 fc_status fc_kv_importance(const void* q, const void* k, fc_dtype dtype, int H, int Lq, int Lk,
                            int d, float scale, float* imp, void* ws, size_t ws_bytes,
                            void* stream) {
+  NvtxRange _range("fc_kv_importance");
   fc::g_launches = 0;
   fc_status st = check_kv_shape(dtype, H, Lq, Lk, d);
   if (st != FC_OK) return st;
@@ -327,6 +344,7 @@ size_t fc_redundancy_workspace_size(fc_dtype dtype, int H, int Lk, int d) {
 
 fc_status fc_kv_redundancy(const void* k, fc_dtype dtype, int H, int Lk, int d, float* red,
                            void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange _range("fc_kv_redundancy");
   fc::g_launches = 0;
   fc_status st = check_kv_shape(dtype, H, Lk, Lk, d);
   if (st != FC_OK) return st;
@@ -349,6 +367,7 @@ size_t fc_score_topb_workspace_size(int H, int Lk, int B) {
 fc_status fc_kv_score_topb(const float* imp, const float* red, int H, int Lk, int pool_window,
                            float lambda, int B, float* score, int32_t* idx, void* ws,
                            size_t ws_bytes, void* stream) {
+  NvtxRange _range("fc_kv_score_topb");
   fc::g_launches = 0;
   if (H < 1 || H > 65535 || Lk < 1) return fail(FC_ERR_INVALID_ARG, "H and Lk must be >= 1");
   if (B < 1) return fail(FC_ERR_INVALID_ARG, "B must be >= 1 (got %d)", B);
@@ -370,6 +389,7 @@ fc_status fc_kv_score_topb(const float* imp, const float* red, int H, int Lk, in
 
 fc_status fc_kv_compact(const void* k, const void* v, fc_dtype dtype, int H, int Lk, int d,
                         const int32_t* idx, int B, void* k_out, void* v_out, void* stream) {
+  NvtxRange _range("fc_kv_compact");
   fc::g_launches = 0;
   fc_status st = check_kv_shape(dtype, H, Lk, Lk, d);
   if (st != FC_OK) return st;
@@ -401,6 +421,7 @@ fc_status fc_kv_cache_commit(const void* q, const void* k_buf, const void* v_buf
                              int C, int n_clean, float scale, int pool_window, float lambda,
                              int32_t* idx, void* ws, size_t ws_bytes, int* n_next,
                              int* compressed, void* stream) {
+  NvtxRange _range("fc_kv_cache_commit");
   fc::g_launches = 0;
   if (n_next == nullptr || compressed == nullptr)
     return fail(FC_ERR_INVALID_ARG, "n_next and compressed must be host pointers");
