@@ -94,12 +94,38 @@ __global__ void __launch_bounds__(kMoveThreads)
                    const int32_t* __restrict__ count, int n_c, int64_t N,
                    float* __restrict__ v_cache) {
   const int slot = blockIdx.y;
+  const int64_t lo = (int64_t)blockIdx.x * kMoveTile, hi = min(N, lo + kMoveTile);
+  if (lo >= hi) return;
+  const float* src = v_dense + (size_t)slot * N;
+  const bool vec = (N & 3) == 0 && ((reinterpret_cast<uintptr_t>(v_dense) |
+                                     reinterpret_cast<uintptr_t>(v_cache)) & 15) == 0;
+  if (vec) {
+    // Whole 16-byte rows: the source tile is loaded before count and ids are
+    // read (the slot's source row is known), so those dependent loads do not
+    // hold up the stream; nothing is written before the slot is known valid.
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+    const int64_t l4 = lo >> 2, h4 = hi >> 2;
+    float4 buf[kMoveVec];
+#pragma unroll
+    for (int u = 0; u < kMoveVec; ++u) {
+      const int64_t i = l4 + threadIdx.x + (int64_t)u * kMoveThreads;
+      if (i < h4) buf[u] = __ldcs(s4 + i);
+    }
+    if (slot >= *count) return;
+    const int dst = ids[slot];
+    if (dst < 0 || dst >= n_c) return;
+    float4* d4 = reinterpret_cast<float4*>(v_cache + (size_t)dst * N);
+#pragma unroll
+    for (int u = 0; u < kMoveVec; ++u) {
+      const int64_t i = l4 + threadIdx.x + (int64_t)u * kMoveThreads;
+      if (i < h4) d4[i] = buf[u];
+    }
+    return;
+  }
   if (slot >= *count) return;
   const int dst = ids[slot];
   if (dst < 0 || dst >= n_c) return;
-  const int64_t lo = (int64_t)blockIdx.x * kMoveTile, hi = min(N, lo + kMoveTile);
-  if (lo >= hi) return;
-  copy_range(v_dense + (size_t)slot * N, v_cache + (size_t)dst * N, N, lo, hi);
+  copy_range(src, v_cache + (size_t)dst * N, N, lo, hi);
 }
 }  // namespace
 
