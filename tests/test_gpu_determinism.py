@@ -82,3 +82,38 @@ def test_cache_commit_is_bitwise_repeatable():
         outs.append([t.cpu() for t in (kn, vn, idx)])
     for p, r in zip(*outs):
         assert torch.equal(p.view(torch.uint8), r.view(torch.uint8))
+
+
+def test_step_soak_replays_bitwise():
+    """The bench's one-layer step (gate and redundancy on a second stream
+    beside the importance) captured once and replayed 200 times: every replay
+    gives the first replay's outputs bitwise, and no bounded wait gives up."""
+    import bench
+
+    dev = torch.device(DEV, torch.cuda.current_device())
+    kv_cfg, gate_cfg = bench.configs("bf16_layer")
+    step = bench.Step(kv_cfg, gate_cfg, seed=0, dev=dev)
+    main = torch.cuda.Stream(device=dev)
+    side = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(main):
+        step.run(main, side=side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=main, capture_error_mode="relaxed"):
+            step.run(main, side=side)
+        names = ("imp", "red", "idx", "ko", "vo")
+        first = None
+        for i in range(200):
+            step.d["x"].copy_(step.host["x"].to(dev))  # the gate updates X in place
+            step.d["f"].zero_()
+            g.replay()
+            main.synchronize()
+            if i % 20 == 0 or i == 199:
+                cur = [step.out[n].clone() for n in names] + [step.d["x"].clone()]
+                if first is None:
+                    first = cur
+                else:
+                    for a, b in zip(first, cur):
+                        assert torch.equal(a.view(torch.uint8), b.view(torch.uint8)), f"replay {i}"
+        del g
+    assert fc.fc_check_workspace(fc.FC_WS_IMPORTANCE, step.ws["imp"])
