@@ -67,7 +67,7 @@ def _args():
     ap.add_argument("--shard", default="layers", choices=["layers", "heads"])
     ap.add_argument("--serial", action="store_true",
                     help="run the five calls one after another on one stream")
-    ap.add_argument("--cpu-sample-heads", type=int, default=4)
+    ap.add_argument("--cpu-sample-heads", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-next", action="store_true",
