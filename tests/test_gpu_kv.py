@@ -243,3 +243,21 @@ def test_compression_chain_against_oracle(name, heads):
         for h in heads:
             assert torch.equal(ko[h], k[h].index_select(0, sel[h]))
             assert torch.equal(vo[h], v[h].index_select(0, sel[h]))
+
+
+@pytest.mark.parametrize("d,dtype", [(64, torch.float32), (128, torch.float32),
+                                     (64, torch.bfloat16), (128, torch.bfloat16)])
+def test_redundancy_long_heads_sampled(d, dtype):
+    """L_k >= 65536 takes the four-rows-in-flight variant: rows sum to one and
+    sampled log-ratios match the oracle's brute-force logits."""
+    H, Lk = 2, 70001
+    g = torch.Generator().manual_seed(d)
+    k = (torch.randn(H, Lk, d, generator=g) + 0.3 * torch.randn(H, 1, d, generator=g)).to(dtype)
+    red = redundancy_gpu(k)
+    np.testing.assert_allclose(red.sum(axis=1), 1.0, rtol=1e-5)
+    rng = np.random.default_rng(d)
+    for h in range(H):
+        cols = np.sort(rng.choice(Lk, 24, replace=False))
+        r = O.redundancy_logits_at(f64(k[h:h + 1]), [0] * cols.size, cols)
+        lr = np.log(red[h, cols].astype(np.float64))
+        np.testing.assert_allclose(lr - lr[0], r - r[0], atol=2e-6)
