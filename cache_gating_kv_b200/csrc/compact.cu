@@ -6,6 +6,7 @@
 // are kept in B_budget.
 //
 // A pure HBM gather: k_out[h][r] = k[h][idx[h][r]] and the same for V, the
+// input heads ldk rows apart (L_k, or B_budget + C for a cache buffer) and the
 // output heads ldo rows apart (B for a dense [H][B][d] result, B_budget + C
 // when the kept rows land in the clean region of a cache buffer).  A row
 // of d elements is d*elem/16 lanes of 16-byte vectors; each thread gathers
@@ -22,14 +23,14 @@ constexpr int kCompactUnroll = 4;
 
 template <int LPR>
 __global__ void __launch_bounds__(kCompactThreads)
-    compact_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int Lk, int B,
+    compact_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int Lk, int ldk, int B,
                    int ldo, const int32_t* __restrict__ idx, uint4* __restrict__ ko,
                    uint4* __restrict__ vo) {
   constexpr int RPW = 32 / LPR;
   constexpr int kRowsPerStep = (kCompactThreads / 32) * RPW;
   constexpr int kRowsPerBlock = kRowsPerStep * kCompactUnroll;
   const int h = blockIdx.y;
-  const uint4* src = (blockIdx.z == 0 ? k : v) + (size_t)h * Lk * LPR;
+  const uint4* src = (blockIdx.z == 0 ? k : v) + (size_t)h * ldk * LPR;
   uint4* dst = (blockIdx.z == 0 ? ko : vo) + (size_t)h * ldo * LPR;
   const int32_t* ih = idx + (size_t)h * B;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -53,12 +54,12 @@ __global__ void __launch_bounds__(kCompactThreads)
 }
 
 template <int LPR>
-cudaError_t run(const void* k, const void* v, int H, int Lk, const int32_t* idx, int B,
+cudaError_t run(const void* k, const void* v, int H, int Lk, int ldk, const int32_t* idx, int B,
                 int ldo, void* ko, void* vo, cudaStream_t s) {
   constexpr int kRowsPerBlock = (kCompactThreads / 32) * (32 / LPR) * kCompactUnroll;
   dim3 grid((unsigned)ceil_div(B, kRowsPerBlock), H, 2);
   compact_kernel<LPR><<<grid, kCompactThreads, 0, s>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), Lk, B, ldo, idx,
+      static_cast<const uint4*>(k), static_cast<const uint4*>(v), Lk, ldk, B, ldo, idx,
       static_cast<uint4*>(ko), static_cast<uint4*>(vo));
   add_launches(1);
   return cudaGetLastError();
@@ -67,12 +68,13 @@ cudaError_t run(const void* k, const void* v, int H, int Lk, const int32_t* idx,
 
 cudaError_t launch_compact(const void* k, const void* v, int elem_bytes, int H, int Lk, int d,
                            const int32_t* idx, int B, int ldo, void* k_out, void* v_out,
-                           cudaStream_t s) {
+                           cudaStream_t s, int ldk) {
+  if (ldk <= 0) ldk = Lk;
   const int row_bytes = d * elem_bytes;
   switch (row_bytes / 16) {
-    case 8: return run<8>(k, v, H, Lk, idx, B, ldo, k_out, v_out, s);
-    case 16: return run<16>(k, v, H, Lk, idx, B, ldo, k_out, v_out, s);
-    case 32: return run<32>(k, v, H, Lk, idx, B, ldo, k_out, v_out, s);
+    case 8: return run<8>(k, v, H, Lk, ldk, idx, B, ldo, k_out, v_out, s);
+    case 16: return run<16>(k, v, H, Lk, ldk, idx, B, ldo, k_out, v_out, s);
+    case 32: return run<32>(k, v, H, Lk, ldk, idx, B, ldo, k_out, v_out, s);
     default: return cudaErrorInvalidValue;
   }
 }

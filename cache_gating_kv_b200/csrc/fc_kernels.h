@@ -34,8 +34,10 @@ cudaError_t launch_scatter_velocity(const float* v_dense, const int32_t* ids, co
 // ---- importance --------------------------------------------------------------
 size_t importance_ws_bytes(int H, int Lq);
 // bf16 tensor-core path (tcgen05 + TMEM + TMA)
+// ldk (here and below): rows between consecutive heads of k (and v); <= 0
+// means Lk (dense heads).  Only the first Lk rows of a head are read.
 cudaError_t launch_importance_tc(const void* q, const void* k, int H, int Lq, int Lk, int d,
-                                 float scale, float* imp, void* ws, cudaStream_t s);
+                                 float scale, float* imp, void* ws, cudaStream_t s, int ldk = 0);
 bool importance_tc_supported(int d);
 // A bounded mbarrier wait that nothing completes, for the self-test
 cudaError_t launch_wait_selftest(long long limit_cycles, int* err, cudaStream_t s);
@@ -45,12 +47,12 @@ cudaError_t launch_exp2_selftest(const float* x, float* y_mufu, float* y_poly, i
 // CUDA-core path (float32 or bf16 inputs)
 cudaError_t launch_importance_simt(const void* q, const void* k, bool bf16, int H, int Lq,
                                    int Lk, int d, float scale, float* imp, void* ws,
-                                   cudaStream_t s);
+                                   cudaStream_t s, int ldk = 0);
 
 // ---- redundancy ----------------------------------------------------------------
 size_t redundancy_ws_bytes(int H, int d);
 cudaError_t launch_redundancy(const void* k, bool bf16, int H, int Lk, int d, float* red,
-                              void* ws, cudaStream_t s);
+                              void* ws, cudaStream_t s, int ldk = 0);
 
 // ---- score + top-B ---------------------------------------------------------------
 size_t score_topb_ws_bytes(int H, int Lk);
@@ -61,6 +63,6 @@ cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk,
 // ---- compaction ------------------------------------------------------------------
 cudaError_t launch_compact(const void* k, const void* v, int elem_bytes, int H, int Lk, int d,
                            const int32_t* idx, int B, int ldo, void* k_out, void* v_out,
-                           cudaStream_t s);
+                           cudaStream_t s, int ldk = 0);
 
 }  // namespace fc

@@ -431,11 +431,8 @@ fc_status fc_kv_cache_commit(const void* q, const void* k_buf, const void* v_buf
   const int cap = B_budget + C;
   fc_status st = check_kv_shape(dtype, H, Lq, cap, d);
   if (st != FC_OK) return st;
-  if (B_budget % C != 0)
-    return fail(FC_ERR_UNSUPPORTED, "B_budget (%d) must be a multiple of C (%d)", B_budget, C);
-  if (n_clean < 0 || n_clean > B_budget || n_clean % C != 0)
-    return fail(FC_ERR_INVALID_ARG, "n_clean must be a multiple of C in [0, B_budget] (got %d)",
-                n_clean);
+  if (n_clean < 0 || n_clean > B_budget)
+    return fail(FC_ERR_INVALID_ARG, "n_clean must be in [0, B_budget] (got %d)", n_clean);
   if (pool_window < 1 || pool_window % 2 == 0 || pool_window > 511)
     return fail(FC_ERR_INVALID_ARG, "pool_window must be odd and in [1, 511] (got %d)",
                 pool_window);
@@ -468,16 +465,21 @@ fc_status fc_kv_cache_commit(const void* q, const void* k_buf, const void* v_buf
   float* red = reinterpret_cast<float*>(w + lay.red);
   int32_t* sel = idx != nullptr ? idx : reinterpret_cast<int32_t*>(w + lay.idx);
   const bool bf16 = dtype == FC_BF16;
-  cudaError_t e = (bf16 && fc::importance_tc_supported(d))
-                      ? fc::launch_importance_tc(q, k_buf, H, Lq, cap, d, scale, imp, w, s)
-                      : fc::launch_importance_simt(q, k_buf, bf16, H, Lq, cap, d, scale, imp, w, s);
-  if (e == cudaSuccess) e = fc::launch_redundancy(k_buf, bf16, H, cap, d, red, w + lay.red_ws, s);
+  // The candidates are the first n_clean + C rows of each head; the heads are
+  // cap rows apart.
+  const int L = n_clean + C;
+  cudaError_t e =
+      (bf16 && fc::importance_tc_supported(d))
+          ? fc::launch_importance_tc(q, k_buf, H, Lq, L, d, scale, imp, w, s, cap)
+          : fc::launch_importance_simt(q, k_buf, bf16, H, Lq, L, d, scale, imp, w, s, cap);
   if (e == cudaSuccess)
-    e = fc::launch_score_topb(imp, red, H, cap, pool_window, lambda, B_budget, nullptr, sel,
+    e = fc::launch_redundancy(k_buf, bf16, H, L, d, red, w + lay.red_ws, s, cap);
+  if (e == cudaSuccess)
+    e = fc::launch_score_topb(imp, red, H, L, pool_window, lambda, B_budget, nullptr, sel,
                               w + lay.score_ws, s);
   if (e == cudaSuccess)
-    e = fc::launch_compact(k_buf, v_buf, (int)elem_bytes(dtype), H, cap, d, sel, B_budget, cap,
-                           k_next, v_next, s);
+    e = fc::launch_compact(k_buf, v_buf, (int)elem_bytes(dtype), H, L, d, sel, B_budget, cap,
+                           k_next, v_next, s, cap);
   st = launched(e, "fc_kv_cache_commit");
   if (st == FC_OK) {
     *n_next = B_budget;

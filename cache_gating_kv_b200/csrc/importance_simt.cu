@@ -69,7 +69,8 @@ __device__ __forceinline__ void tile_dot(const float* __restrict__ As, const flo
 
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
-    imp_lse_simt(const T* __restrict__ q, const T* __restrict__ k, int Lq, int Lk, float c2,
+    imp_lse_simt(const T* __restrict__ q, const T* __restrict__ k, int Lq, int Lk, int ldk,
+                 float c2,
                  float* __restrict__ lse2) {
   extern __shared__ __align__(16) float sm[];
   float* Qs = sm;
@@ -85,7 +86,7 @@ __global__ void __launch_bounds__(kThreads)
   }
   for (int k0 = 0; k0 < Lk; k0 += kT) {
     __syncthreads();
-    load_tile_t<T, D>(Ks, k + ((size_t)h * Lk + k0) * D, min(kT, Lk - k0));
+    load_tile_t<T, D>(Ks, k + ((size_t)h * ldk + k0) * D, min(kT, Lk - k0));
     __syncthreads();
     float acc[4][4];
     tile_dot<D>(Qs, Ks, ty, tx, acc);
@@ -131,14 +132,14 @@ __global__ void __launch_bounds__(kThreads)
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
     imp_col_simt(const T* __restrict__ q, const T* __restrict__ k, const float* __restrict__ lse2,
-                 int Lq, int Lk, float c2, float* __restrict__ imp) {
+                 int Lq, int Lk, int ldk, float c2, float* __restrict__ imp) {
   extern __shared__ __align__(16) float sm[];
   float* Ks = sm;
   float* Qs = sm + D * kPad;
   float* sl = sm + 2 * D * kPad;  // [64] row normalisers of the query tile
   const int h = blockIdx.y, k0 = blockIdx.x * kT;
   const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
-  load_tile_t<T, D>(Ks, k + ((size_t)h * Lk + k0) * D, min(kT, Lk - k0));
+  load_tile_t<T, D>(Ks, k + ((size_t)h * ldk + k0) * D, min(kT, Lk - k0));
   float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   for (int q0 = 0; q0 < Lq; q0 += kT) {
     __syncthreads();
@@ -172,7 +173,7 @@ __global__ void __launch_bounds__(kThreads)
 }
 
 template <typename T, int D>
-cudaError_t run(const T* q, const T* k, int H, int Lq, int Lk, float scale, float* imp,
+cudaError_t run(const T* q, const T* k, int H, int Lq, int Lk, int ldk, float scale, float* imp,
                 float* lse2, cudaStream_t s) {
   const float c2 = scale * kLog2e;
   const size_t smem1 = (size_t)2 * D * kPad * sizeof(float);
@@ -182,27 +183,29 @@ cudaError_t run(const T* q, const T* k, int H, int Lq, int Lk, float scale, floa
   cudaFuncSetAttribute(imp_col_simt<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)smem2);
   imp_lse_simt<T, D><<<dim3((unsigned)ceil_div(Lq, kT), H), kThreads, smem1, s>>>(q, k, Lq, Lk,
-                                                                                  c2, lse2);
+                                                                                  ldk, c2, lse2);
   imp_col_simt<T, D><<<dim3((unsigned)ceil_div(Lk, kT), H), kThreads, smem2, s>>>(
-      q, k, lse2, Lq, Lk, c2, imp);
+      q, k, lse2, Lq, Lk, ldk, c2, imp);
   add_launches(2);
   return cudaGetLastError();
 }
 }  // namespace
 
 cudaError_t launch_importance_simt(const void* q, const void* k, bool bf16, int H, int Lq, int Lk,
-                                   int d, float scale, float* imp, void* ws, cudaStream_t s) {
+                                   int d, float scale, float* imp, void* ws, cudaStream_t s,
+                                   int ldk) {
+  if (ldk <= 0) ldk = Lk;
   float* lse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + 256);  // after the error word
   if (bf16) {
     const auto* qb = static_cast<const __nv_bfloat16*>(q);
     const auto* kb = static_cast<const __nv_bfloat16*>(k);
-    return d == 128 ? run<__nv_bfloat16, 128>(qb, kb, H, Lq, Lk, scale, imp, lse2, s)
-                    : run<__nv_bfloat16, 64>(qb, kb, H, Lq, Lk, scale, imp, lse2, s);
+    return d == 128 ? run<__nv_bfloat16, 128>(qb, kb, H, Lq, Lk, ldk, scale, imp, lse2, s)
+                    : run<__nv_bfloat16, 64>(qb, kb, H, Lq, Lk, ldk, scale, imp, lse2, s);
   }
   const auto* qf = static_cast<const float*>(q);
   const auto* kf = static_cast<const float*>(k);
-  return d == 128 ? run<float, 128>(qf, kf, H, Lq, Lk, scale, imp, lse2, s)
-                  : run<float, 64>(qf, kf, H, Lq, Lk, scale, imp, lse2, s);
+  return d == 128 ? run<float, 128>(qf, kf, H, Lq, Lk, ldk, scale, imp, lse2, s)
+                  : run<float, 64>(qf, kf, H, Lq, Lk, ldk, scale, imp, lse2, s);
 }
 
 }  // namespace fc

@@ -417,11 +417,13 @@ EncodeTiledFn encode_fn() {
 }
 
 // [H][L][d] bf16, box = 64 elements (128 B, the swizzle span) x `rows` x 1 head.
-bool make_map(CUtensorMap* map, const void* ptr, int H, int L, int d, int rows) {
+// Tensor map over [H][L][d] bf16 whose heads are `ld` rows apart (ld >= L);
+// rows past L read as zero.
+bool make_map(CUtensorMap* map, const void* ptr, int H, int L, int d, int rows, int ld) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)L, (cuuint64_t)H};
-  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)L * d * 2};
+  const cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)ld * d * 2};
   const cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
@@ -431,12 +433,12 @@ bool make_map(CUtensorMap* map, const void* ptr, int H, int L, int d, int rows) 
 }
 
 template <int D>
-cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, float scale, float* imp,
-                void* ws, cudaStream_t s) {
+cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, int ldk, float scale,
+                float* imp, void* ws, cudaStream_t s) {
   // A operands are 128-row tiles, B operands 256-row tiles.
   CUtensorMap mqA, mqB, mkA, mkB;
-  if (!make_map(&mqA, q, H, Lq, D, kBM) || !make_map(&mqB, q, H, Lq, D, kBN) ||
-      !make_map(&mkA, k, H, Lk, D, kBM) || !make_map(&mkB, k, H, Lk, D, kBN))
+  if (!make_map(&mqA, q, H, Lq, D, kBM, Lq) || !make_map(&mqB, q, H, Lq, D, kBN, Lq) ||
+      !make_map(&mkA, k, H, Lk, D, kBM, ldk) || !make_map(&mkB, k, H, Lk, D, kBN, ldk))
     return cudaErrorInvalidValue;
   int* err = reinterpret_cast<int*>(static_cast<char*>(ws) + kErrOffset);
   const int lq_pad = (int)ceil_div(Lq, kBN) * kBN;
@@ -510,9 +512,10 @@ size_t importance_ws_bytes(int H, int Lq) {
 bool importance_tc_supported(int d) { return d == 64 || d == 128; }
 
 cudaError_t launch_importance_tc(const void* q, const void* k, int H, int Lq, int Lk, int d,
-                                 float scale, float* imp, void* ws, cudaStream_t s) {
-  return d == 128 ? run<128>(q, k, H, Lq, Lk, scale, imp, ws, s)
-                  : run<64>(q, k, H, Lq, Lk, scale, imp, ws, s);
+                                 float scale, float* imp, void* ws, cudaStream_t s, int ldk) {
+  if (ldk <= 0) ldk = Lk;
+  return d == 128 ? run<128>(q, k, H, Lq, Lk, ldk, scale, imp, ws, s)
+                  : run<64>(q, k, H, Lq, Lk, ldk, scale, imp, ws, s);
 }
 
 cudaError_t launch_exp2_selftest(const float* x, float* y_mufu, float* y_poly, int n,

@@ -88,7 +88,7 @@ __device__ __forceinline__ void unpack(const uint4 (&u)[2], float* e) {
 // U: rows in flight per lane (two 16-byte loads each).
 template <typename T, int D, int U>
 __global__ void __launch_bounds__(kRedThreads)
-    red_cluster_kernel(const T* __restrict__ k, int Lk, int h0, float* __restrict__ red) {
+    red_cluster_kernel(const T* __restrict__ k, int Lk, int ldk, int h0, float* __restrict__ red) {
   using L = RowLayout<T, D>;
   cg::cluster_group cluster = cg::this_cluster();
   const int nrank = (int)cluster.num_blocks();
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(kRedThreads)
   const int sub = lane / L::LPR, cl = lane % L::LPR;
   const int per = (int)ceil_div(Lk, nrank);
   const int lo = min(Lk, rank * per), hi = min(Lk, lo + per);
-  const T* kh = k + (size_t)h * Lk * D;
+  const T* kh = k + (size_t)h * ldk * D;
   constexpr int kRowsPerIter = kRedWarps * L::RPW * U;
 
   __shared__ float s_acc[kRedWarps][D];
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(kRedThreads)
 }
 
 template <typename T, int D>
-cudaError_t run(const T* k, int H, int Lk, float* red, cudaStream_t s) {
+cudaError_t run(const T* k, int H, int Lk, int ldk, float* red, cudaStream_t s) {
   // 16 CTAs per head when the slices stay long enough, else the portable 8.
   const int csize = (Lk >= 16 * 64) ? 16 : 8;
   // Long heads keep four rows per lane in flight (two measured 17 % slower at
@@ -233,7 +233,7 @@ cudaError_t run(const T* k, int H, int Lk, float* red, cudaStream_t s) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, k, Lk, 0, red);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, k, Lk, ldk, 0, red);
   if (e != cudaSuccess) return e;
   add_launches(1);
   return cudaSuccess;
@@ -247,15 +247,16 @@ size_t redundancy_ws_bytes(int H, int d) {
 }
 
 cudaError_t launch_redundancy(const void* k, bool bf16, int H, int Lk, int d, float* red,
-                              void* ws, cudaStream_t s) {
+                              void* ws, cudaStream_t s, int ldk) {
   (void)ws;
+  if (ldk <= 0) ldk = Lk;
   if (bf16) {
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
-    return d == 128 ? run<__nv_bfloat16, 128>(kb, H, Lk, red, s)
-                    : run<__nv_bfloat16, 64>(kb, H, Lk, red, s);
+    return d == 128 ? run<__nv_bfloat16, 128>(kb, H, Lk, ldk, red, s)
+                    : run<__nv_bfloat16, 64>(kb, H, Lk, ldk, red, s);
   }
   const float* kf = static_cast<const float*>(k);
-  return d == 128 ? run<float, 128>(kf, H, Lk, red, s) : run<float, 64>(kf, H, Lk, red, s);
+  return d == 128 ? run<float, 128>(kf, H, Lk, ldk, red, s) : run<float, 64>(kf, H, Lk, ldk, red, s);
 }
 
 }  // namespace fc

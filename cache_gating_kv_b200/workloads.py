@@ -152,6 +152,12 @@ CACHE_CONFIGS = {
     # 4 heads, d=128, chunks of 1024 tokens, budget 4 chunks, 8 chunks, bf16.
     "bf16_stream": CacheConfig("bf16_stream", H=4, d=128, C=1024, B_budget=4096, n_chunks=8,
                                Lq=256, lam=0.5, pool=7, dtype="bf16", rho=0.95),
+    # Chunk sizes that do not divide the budget: the first compression scores
+    # fewer than B_budget + C candidates.
+    "tiny_fp32_ragged": CacheConfig("tiny_fp32_ragged", H=2, d=64, C=37, B_budget=100,
+                                    n_chunks=7, Lq=40, lam=0.5, pool=3, dtype="f32", rho=0.9),
+    "bf16_ragged": CacheConfig("bf16_ragged", H=3, d=128, C=300, B_budget=1000, n_chunks=6,
+                               Lq=96, lam=0.5, pool=7, dtype="bf16", rho=0.95),
 }
 
 

@@ -349,8 +349,9 @@ size_t fc_kv_cache_workspace_size(fc_dtype dtype, int H, int Lq, int B_budget, i
  *   - If n_clean + C <= B_budget the chunk is kept where it is: *n_next =
  *     n_clean + C, *compressed = 0, nothing is launched and no device pointer
  *     is read (they may be NULL).
- *   - Otherwise the cap candidates are scored as fc_kv_importance (queries q),
- *     fc_kv_redundancy and fc_kv_score_topb with B = B_budget would score them,
+ *   - Otherwise the n_clean + C candidates (n_clean + C <= cap) are scored as
+ *     fc_kv_importance (queries q), fc_kv_redundancy and fc_kv_score_topb with
+ *     B = B_budget would score them,
  *     and the kept rows of every head are written once, in candidate order, to
  *     rows [0, B_budget) of the other buffer (k_next, v_next); rows
  *     [B_budget, cap) of that buffer are not written (the next chunk's K/V go
@@ -361,17 +362,16 @@ size_t fc_kv_cache_workspace_size(fc_dtype dtype, int H, int Lq, int B_budget, i
  *   k_next, v_next [H][cap][d] dtype, the other buffer; no overlap with the
  *                  current one or with each other
  *   d              64 or 128
- *   C              tokens per chunk, >= 1; B_budget a multiple of C (so a
- *                  compression always sees exactly cap candidates)
- *   n_clean        a multiple of C in [0, B_budget]
+ *   C              tokens per chunk, 1 <= C <= B_budget
+ *   n_clean        clean rows in [0, B_budget]
  *   scale          softmax scale, <= 0 means 1/sqrt(d)
  *   pool_window, lambda  as for fc_kv_score_topb
  *   idx            [H][B_budget] int32 out (the kept candidate rows,
  *                  ascending), or NULL to keep them in the workspace only
  *   n_next, compressed   host ints, out
  * Errors: bad sizes or pointers, overlapping buffers -> FC_ERR_INVALID_ARG;
- * B_budget not a multiple of C, d not 64/128 -> FC_ERR_UNSUPPORTED; small
- * ws -> FC_ERR_WORKSPACE.  On an error *n_next and *compressed are unchanged.
+ * d not 64/128 -> FC_ERR_UNSUPPORTED; small ws -> FC_ERR_WORKSPACE.  On an
+ * error *n_next and *compressed are unchanged.
  */
 fc_status fc_kv_cache_commit(const void* q, const void* k_buf, const void* v_buf, void* k_next,
                              void* v_next, fc_dtype dtype, int H, int Lq, int d, int B_budget,

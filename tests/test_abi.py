@@ -162,11 +162,15 @@ def test_cache_commit_validates_and_keeps_fitting_chunks_on_the_host():
     assert lib.fc_last_launches() == 0
     n_next.value = comp.value = -1
     assert commit(B=96, C=96, n=0) == 0 and (n_next.value, comp.value) == (96, 0)
-    # B_budget not a multiple of C; d unsupported
-    assert commit(B=100, C=32) == 2
+    # any chunk size: B_budget need not be a multiple of C, n_clean any count
+    n_next.value = comp.value = -1
+    assert commit(B=100, C=32, n=68) == 0 and (n_next.value, comp.value) == (100, 0)
+    assert commit(n=16) == 0 and (n_next.value, comp.value) == (48, 0)
+    assert lib.fc_last_launches() == 0
+    # d unsupported
     assert commit(d=96) == 2
-    # n_clean not a multiple of C, out of range, C < 1, C > B_budget, even window
-    assert commit(n=16) == 1
+    # n_clean out of range, C < 1, C > B_budget, even window
+    assert commit(n=-1) == 1
     assert commit(n=128) == 1
     assert commit(C=0) == 1
     assert commit(C=128) == 1

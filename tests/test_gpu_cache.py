@@ -9,7 +9,11 @@ compression) with the oracle's cache_commit / cache_stream.
 - bf16 stream: every commit equals the separate calls (importance,
   redundancy, score/top-B, compaction) on the same buffer, bitwise;
 - bf16 stream with lambda = 1, no pooling and one query repeated: the final
-  clean set is the global top-B_budget by q.k (brute force in float64)."""
+  clean set is the global top-B_budget by q.k (brute force in float64);
+- streams whose chunk size does not divide the budget (both dtypes): the
+  clean counts follow the oracle's, every compression selects under the
+  margin waiver from exactly the n_clean + C candidates (the buffer rows past
+  them are NaN) and keeps those rows bitwise."""
 
 import numpy as np
 import pytest
@@ -205,3 +209,40 @@ def test_bf16_importance_only_keeps_global_top_b():
         sel = torch.from_numpy(pos[h])
         assert torch.equal(gk[h], allk[h].index_select(0, sel))
         assert torch.equal(gv[h], allv[h].index_select(0, sel))
+
+
+@pytest.mark.parametrize("name", ["tiny_fp32_ragged", "bf16_ragged"])
+def test_ragged_chunk_stream(name):
+    cfg = W.CACHE_CONFIGS[name]
+    ks, vs, qs = W.cache_inputs(cfg, seed=4)
+    H, C, B, d = cfg.H, cfg.C, cfg.B_budget, cfg.d
+    bf16 = cfg.dtype == "bf16"
+    dtype = torch.bfloat16 if bf16 else torch.float32
+    tol = TOL_BF16 if bf16 else TOL_F32
+    g = GpuCache(H, C, B, d, cfg.Lq, dtype, sentinel=float("nan"))
+    n_ref = 0
+    sizes = []
+    for i in range(cfg.n_chunks):
+        g.write_chunk(ks[i], vs[i])
+        L = g.n + C
+        kb0, vb0 = (t[:, :L].cpu() for t in g.bufs[g.cur])
+        comp = g.commit(qs[i], cfg.lam, cfg.pool)
+        # the oracle's clean count for the same stream
+        n_ref = n_ref + C if n_ref + C <= B else B
+        assert g.n == n_ref and comp == (L > B)
+        if not comp:
+            continue
+        sizes.append(L)
+        idx = g.idx.cpu().numpy()
+        assert idx.min() >= 0 and idx.max() < L
+        kc = f64(kb0)
+        sc = O.score(O.importance(f64(qs[i]), kc), O.redundancy(kc), cfg.lam, cfg.pool)
+        kn, vn = g.bufs[g.cur]
+        for h in range(H):
+            span = (sc[h].max() - sc[h].min()) if bf16 else np.abs(sc[h]).max()
+            assert_selection_matches(idx[h:h + 1], sc[h:h + 1], B, tol * max(float(span), 1e-30))
+            sel = torch.from_numpy(idx[h].astype(np.int64))
+            assert torch.equal(kn[h, :B].cpu(), kb0[h].index_select(0, sel))
+            assert torch.equal(vn[h, :B].cpu(), vb0[h].index_select(0, sel))
+    # the first compression saw fewer than B_budget + C candidates, the rest all of them
+    assert sizes[0] < B + C and all(s == B + C for s in sizes[1:]) and len(sizes) >= 2

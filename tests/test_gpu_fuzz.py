@@ -134,30 +134,38 @@ def test_history_gate_random(seed):
 
 @pytest.mark.parametrize("seed", range(16))
 def test_cache_commit_random(seed):
-    """One compression of a full float32 cache buffer with random sizes."""
+    """One compression of a float32 cache buffer with random sizes: B_budget
+    any multiple of C or not, n_clean any count that makes the chunk overflow,
+    the buffer rows past the n_clean + C candidates poisoned with NaN (they
+    must never be read)."""
     rng = np.random.default_rng(11000 + seed)
     H = int(rng.integers(1, 4))
     d = int(rng.choice([64, 128]))
     C = int(rng.integers(1, 200))
-    B = C * int(rng.integers(1, 5))
+    B = C * int(rng.integers(1, 5)) if seed % 2 == 0 else int(rng.integers(C, 4 * C + 1))
+    n = B if seed % 4 < 2 else int(rng.integers(max(B - C + 1, 0), B + 1))
+    L = n + C
     Lq = int(rng.integers(1, 300))
     pool = int(rng.choice([1, 3, 7]))
     lam = float(rng.uniform(0.0, 1.0))
     g = torch.Generator().manual_seed(seed)
-    kb = torch.randn(H, B + C, d, generator=g)
-    vb = torch.randn(H, B + C, d, generator=g)
+    kb = torch.full((H, B + C, d), float("nan"))
+    vb = torch.full((H, B + C, d), float("nan"))
+    kb[:, :L] = torch.randn(H, L, d, generator=g)
+    vb[:, :L] = torch.randn(H, L, d, generator=g)
     q = torch.randn(H, Lq, d, generator=g)
     kn = torch.full_like(kb, 5.0).to(DEV)
     vn = torch.full_like(vb, 5.0).to(DEV)
     ws = fc.workspace(fc.fc_kv_cache_workspace_size(fc.FC_F32, H, Lq, B, C, d))
     idx = torch.empty(H, B, dtype=torch.int32, device=DEV)
-    n, comp = fc.fc_kv_cache_commit(q.to(DEV), kb.to(DEV), vb.to(DEV), kn, vn, B, C, ws, pool,
-                                    lam, idx=idx)
+    n_next, comp = fc.fc_kv_cache_commit(q.to(DEV), kb.to(DEV), vb.to(DEV), kn, vn, n, C, ws,
+                                         pool, lam, idx=idx)
     torch.cuda.synchronize()
-    assert comp and n == B
-    kc = f64(kb)
+    assert comp and n_next == B
+    kc = f64(kb[:, :L])
     sc_r = O.score(O.importance(f64(q), kc), O.redundancy(kc), lam, pool)
     gi = idx.cpu().numpy()
+    assert gi.min() >= 0 and gi.max() < L
     for h in range(H):
         span = max(float(np.abs(sc_r[h]).max()), 1e-30)
         assert_selection_matches(gi[h:h + 1], sc_r[h:h + 1].astype(np.float64), B, TOL_F32 * span)

@@ -480,12 +480,32 @@ def test_cache_fills_then_holds_the_budget():
     np.testing.assert_array_equal(vb[:, :12], np.concatenate(vs[:3], axis=1))
 
 
-def test_cache_importance_only_keeps_global_top_b_by_dot_product():
+def test_cache_ragged_chunks_fill_to_the_budget():
+    """A chunk size that does not divide the budget: the clean length grows by
+    C while n + C fits, the first overflow compresses n + C < B + C candidates
+    down to B, and from then on every chunk brings B + C candidates."""
+    H, C, d, B = 2, 5, 8, 12
+    ks, vs, qs = _stream_inputs(H, C, d, 6, 3, seed=2)
+    _, _, n, lengths = O.cache_stream(ks, vs, qs, B, 0.5, 3)
+    assert lengths == [5, 10, 12, 12, 12, 12] and n == 12
+    kb = np.zeros((H, B + C, d))
+    vb = np.zeros((H, B + C, d))
+    kb[:, :15] = np.concatenate(ks[:3], axis=1)
+    vb[:, :15] = np.concatenate(vs[:3], axis=1)
+    kn, vn, n, idx = O.cache_commit(kb, vb, 10, C, B, qs[2], 0.5, 3)
+    assert n == 12 and idx.shape == (H, 12) and idx.max() < 15
+    for h in range(H):
+        np.testing.assert_array_equal(kn[h, :12], kb[h, idx[h]])
+
+
+@pytest.mark.parametrize("C,B", [(4, 8), (3, 8), (5, 7)])
+def test_cache_importance_only_keeps_global_top_b_by_dot_product(C, B):
     """lambda = 1, no pooling and one query repeated: the softmax is monotone
     in q.k, so each compression keeps the B largest q.k among its candidates,
     and over the stream the clean set is the B largest q.k of all tokens seen,
-    in the order they arrived (brute force over the concatenated tokens)."""
-    H, C, d, B, n_chunks = 3, 4, 8, 8, 6
+    in the order they arrived (brute force over the concatenated tokens).
+    Holds whether or not C divides B."""
+    H, d, n_chunks = 3, 8, 6
     ks, vs, qs = _stream_inputs(H, C, d, n_chunks, 5, seed=1, same_query=True)
     kb, vb, n, _ = O.cache_stream(ks, vs, qs, B, 1.0, 1)
     allk = np.concatenate(ks, axis=1)
