@@ -255,7 +255,7 @@ size_t fc_importance_workspace_size(fc_dtype dtype, int H, int Lq, int Lk, int d
  *          word that the tensor-core path sets to nonzero if one of its
  *          bounded device-side waits gave up (the call never clears it; zero
  *          it once; read it with fc_check_workspace); the per-query log-sum-exp
- *          follows from byte 256
+ *          normalisers (split into bf16 terms) follow from byte 256
  * Errors: H, Lq, Lk < 1 or d not in {64, 128} -> FC_ERR_INVALID_ARG /
  * FC_ERR_UNSUPPORTED; bad pointers -> FC_ERR_INVALID_ARG; small ws ->
  * FC_ERR_WORKSPACE.
