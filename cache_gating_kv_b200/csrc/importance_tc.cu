@@ -6,12 +6,12 @@
 //
 // The L_q x L_k probability matrix is never stored.  Two passes recompute the
 // logits with tcgen05.mma:
-//   pass 1 (rows)     CTA = 128 queries of one head; streams every 256-key
+//   pass 1 (rows)     CTA = 256 queries of one head; streams every 256-key
 //                     tile; D = Q K^T in TMEM; the epilogue thread that owns a
 //                     query row keeps a (reference, sum) pair in log2 units
 //                     and the CTA writes nl_q = -log2 sum_j 2^(c s_qj),
 //                     c = scale*log2(e) (padded query rows: -inf).
-//   pass 2 (columns)  CTA = 128 keys of one head; streams every 256-query tile;
+//   pass 2 (columns)  CTA = 256 keys of one head; streams every 256-query tile;
 //                     D = K Q^T + nl/c in TMEM (keys on the TMEM lanes), so
 //                     each epilogue thread owns one key and sums 2^(c D)
 //                     over all queries in registers: no atomics, no partial
@@ -33,10 +33,13 @@
 //     reading its operands from shared memory (measured ~1.0 PFLOP/s with the
 //     epilogue and TMA removed); N=256 reuses each A fragment for twice the
 //     columns;
-//   - keeps two 256-column TMEM accumulators in flight and lets every
-//     epilogue warpgroup drain its own 64-column slice of every tile: an
-//     accumulator is handed back to the MMA as soon as each warp has loaded
-//     its slice;
+//   - holds two 128-row A tiles per CTA, each with its own 256-column TMEM
+//     accumulator, and feeds every streamed B tile to both (ping-pong): the
+//     eight epilogue warps of one A tile drain its accumulator (two
+//     warpgroups, 128 columns each) while the MMA for the other tile runs,
+//     and an accumulator is handed back to the MMA as soon as each of its
+//     warps has loaded its slice (measured 1-3 % faster than one A tile with
+//     two accumulators, and each B tile crosses from L2 once per 256 rows);
 //   - uses packed f32x2 FMA/ADD for the scale-and-shift and the running sums;
 //   - evaluates 1 of every 4 exponentials on the FMA pipes (ex2_poly2, a
 //     polynomial of our own) and the rest on the special-function unit (a
@@ -44,6 +47,10 @@
 //   - in pass 1 shifts by a lagged reference instead of the exact running max:
 //     the reference only moves (with an exact rescale) when a chunk's sum
 //     exceeds 2^32, so the per-element max disappears from the common path;
+//     the chunks of a slice fold their overflow tests into one flag, read once
+//     before the accumulator is released, and the rare overflowing slice is
+//     redone from TMEM with the exact per-chunk test (a branch per chunk kept
+//     the next chunk's work from overlapping: 3 % of both passes);
 //   - in pass 1 splits the key range in 2-4 parts when that fills the last
 //     wave of CTAs better; a small kernel merges the partial (reference, sum)
 //     pairs.
@@ -52,8 +59,8 @@
 // [H][L][d], 128-byte swizzle, zero fill past L, no multicast; pass 2 also the
 // [H][Lq_pad][16] extra rows, 32-byte swizzle), warp 1 lane 0
 // issues the MMAs (M=128, N=256, K=16 steps), warp 2 owns the TMEM allocation
-// (all 512 columns), warps 4-19 are four epilogue warpgroups (warp w reads
-// TMEM lanes 32(w%4)..+31).  A two-stage shared-memory ring of 64 KB operand
+// (all 512 columns), warps 4-11 drain A tile 0 and warps 12-19 A tile 1 (warp w
+// reads TMEM lanes 32(w%4)..+31).  A two-stage shared-memory ring of 64 KB operand
 // tiles decouples TMA from the MMAs.  Every mbarrier wait is bounded; on timeout the kernel
 // records an error word in the workspace and winds down (no trap, no endless
 // spin).
@@ -69,18 +76,16 @@ namespace {
 constexpr int kBM = 128;      // rows of the resident A tile (MMA M, TMEM lanes)
 constexpr int kBN = 256;      // rows of each streamed B tile (MMA N, TMEM columns)
 constexpr int kStages = 2;    // shared-memory ring depth (64 KB B tiles)
-constexpr int kAcc = 2;       // TMEM accumulators of kBN columns (all 512 columns)
-#ifndef FC_IMP_EPI
-#define FC_IMP_EPI 4
-#endif
+constexpr int kNA = 2;        // A tiles per CTA, one TMEM accumulator of kBN columns each
 #ifndef FC_IMP_EMU_MASK
 #define FC_IMP_EMU_MASK 0x2222  // pairs 1, 5, 9, 13 of 16: 1/4 of the exponentials
 #endif
-constexpr int kEpi = FC_IMP_EPI;  // epilogue warpgroups; each owns kBN/kEpi columns of every tile
-constexpr int kThreads = 128 + 128 * kEpi;
+constexpr int kWG = 2;        // epilogue warpgroups per A tile; each owns kBN/kWG columns
+constexpr int kEpiWarps = kNA * kWG * 4;
+constexpr int kThreads = 128 + 32 * kEpiWarps;
 constexpr int kCh = 32;       // TMEM columns per tcgen05.ld chunk
-constexpr int kSlice = kBN / kEpi;  // columns of a tile that one epilogue group drains
-static_assert(kSlice % kCh == 0, "each group drains whole chunks");
+constexpr int kSlice = kBN / kWG;  // columns of a tile that one warpgroup drains
+static_assert(kSlice % kCh == 0, "each warpgroup drains whole chunks");
 constexpr int kHalfA = kBM * 64 * 2;  // one 128-row x 64-element bf16 swizzled block (16 KB)
 constexpr int kHalfB = kBN * 64 * 2;  // one 256-row x 64-element bf16 swizzled block (32 KB)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -107,8 +112,8 @@ constexpr int kXBytes = kBN * kXRow;     // pass 2: the query tile's extra block
 constexpr int kOnesBytes = kBM * kXRow;  // pass 2: the key tile's extra block (all ones)
 template <int D>
 constexpr size_t smem_bytes() {
-  return 1024 + (size_t)a_bytes<D>() + (size_t)kStages * b_bytes<D>() +
-         (size_t)kStages * kXBytes + kOnesBytes + 256 + 2 * kEpi * kBM * sizeof(float);
+  return 1024 + (size_t)kNA * a_bytes<D>() + (size_t)kStages * b_bytes<D>() +
+         (size_t)kStages * kXBytes + kOnesBytes + 256 + (size_t)kNA * kWG * 2 * kBM * sizeof(float);
 }
 
 // Row of the extra K block of pass 2 for one query: x = nl / (2 c) split into
@@ -136,13 +141,13 @@ struct Bars {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t a_full;
-  uint64_t acc_full[kAcc];
-  uint64_t acc_empty[kAcc];
+  uint64_t acc_full[kNA];
+  uint64_t acc_empty[kNA];
   uint32_t tmem_slot;
 };
 
 __device__ __forceinline__ void epilogue_sync() {
-  asm volatile("bar.sync 1, %0;" ::"n"(128 * kEpi) : "memory");  // the epilogue warps only
+  asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpiWarps) : "memory");  // the epilogue warps only
 }
 
 __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) {
@@ -202,6 +207,19 @@ __device__ __forceinline__ void row_chunk(uint32_t (&r)[kCh], int valid, float c
   l += cs;
 }
 
+// Pass 1, the rare path: redo the first n chunks of a slice from TMEM with
+// the exact per-chunk check (out of line, so its registers do not weigh on
+// the common path).  Called by all 32 lanes of a warp together (tcgen05.ld
+// and its wait are warp-collective).
+__device__ __noinline__ void redo_chunks(uint32_t addr, int n, float c2, float& ref, float& l) {
+  for (int c = 0; c < n; ++c) {
+    uint32_t r[kCh];
+    tc::tmem_ld32(addr + c * kCh, r);
+    tc::tmem_ld_wait(r);
+    row_chunk(r, kCh, c2, ref, l);
+  }
+}
+
 // Pass 2 on one chunk: acc += 2^(c*(s + nl_q/c)) over the chunk's 32 queries
 // (the MMA already added nl_q/c to every logit).
 __device__ __forceinline__ void col_chunk(const uint32_t (&r)[kCh], float c2, float2& acc) {
@@ -218,8 +236,12 @@ __device__ __forceinline__ void col_chunk(const uint32_t (&r)[kCh], float c2, fl
   acc = tc::fadd2(acc, a1);
 }
 
-// kPass 1: A = Q tile, B = K tiles of one key split, epilogue = row log-sum-exp.
-// kPass 2: A = K tile, B = Q tiles (+ the extra K step), epilogue = column
+// CTA = two A tiles (256 rows) of one head; every streamed B tile feeds two
+// MMAs, one per A tile, each into its own 256-column accumulator.  The eight
+// epilogue warps of A tile j drain accumulator j while the MMA for the other
+// tile runs (ping-pong).
+// kPass 1: A = Q tiles, B = K tiles of one key split, epilogue = row log-sum-exp.
+// kPass 2: A = K tiles, B = Q tiles (+ the extra K step), epilogue = column
 // sums of 2^(c (s + nl/c)).
 template <int D, int kPass>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -234,18 +256,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~(uintptr_t)1023);
-  uint8_t* sA = base;
-  uint8_t* sB = base + TA;
+  uint8_t* sA = base;                        // [kNA] A tiles
+  uint8_t* sB = base + kNA * TA;             // [kStages] B tiles
   uint8_t* sX = sB + kStages * TB;           // pass 2: [kStages][kBN][32 B]
   uint8_t* sOnes = sX + kStages * kXBytes;   // pass 2: [kBM][32 B] of bf16 ones
   Bars* bars = reinterpret_cast<Bars*>(sOnes + kOnesBytes);
-  float* sM = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // [2*kEpi][kBM]
+  float* sM = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // merge buffer
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y;
   const int unit = kPass == 1 ? blockIdx.x / nsplit : blockIdx.x;
   const int split = kPass == 1 ? blockIdx.x % nsplit : 0;
-  const int a0 = unit * kBM;  // first row of the A tile
+  const int a0 = unit * (kNA * kBM);  // first row of the A tiles
   int t_begin = 0, nB;
   if (kPass == 1) {
     const int nkt = (Lk + kBN - 1) / kBN;
@@ -262,13 +284,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_init(&bars->empty[s], 1);
     }
     tc::mbar_init(&bars->a_full, 1);
-    for (int b = 0; b < kAcc; ++b) {
-      tc::mbar_init(&bars->acc_full[b], 1);
-      tc::mbar_init(&bars->acc_empty[b], 4 * kEpi);  // every epilogue warp reads its slice
+    for (int j = 0; j < kNA; ++j) {
+      tc::mbar_init(&bars->acc_full[j], 1);
+      tc::mbar_init(&bars->acc_empty[j], 4 * kWG);  // every warp of tile j reads its slice
     }
     tc::fence_barrier_init();
   }
-  if (warp == 2) tc::tmem_alloc(&bars->tmem_slot, kAcc * kBN);
+  if (warp == 2) tc::tmem_alloc(&bars->tmem_slot, kNA * kBN);
   if (kPass == 2 && threadIdx.x >= 128 && threadIdx.x < 128 + kOnesBytes / 16) {
     reinterpret_cast<uint4*>(sOnes)[threadIdx.x - 128] =
         make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
@@ -282,9 +304,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {  // ---- TMA producer
-      tc::mbar_expect_tx(&bars->a_full, TA);
-      for (int kb = 0; kb < KB; ++kb)
-        tc::tma_load_3d(sA + kb * kHalfA, &mapA, &bars->a_full, kb * 64, a0, h);
+      tc::mbar_expect_tx(&bars->a_full, kNA * TA);
+      for (int j = 0; j < kNA; ++j)
+        for (int kb = 0; kb < KB; ++kb)
+          tc::tma_load_3d(sA + j * TA + kb * kHalfA, &mapA, &bars->a_full, kb * 64,
+                          a0 + j * kBM, h);
       for (int t = 0; t < nB; ++t) {
         const int s = t % kStages, u = t / kStages;
         if (!tc::mbar_wait(&bars->empty[s], (u & 1) ^ 1)) {
@@ -301,55 +325,97 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     if (lane == 0) {  // ---- MMA issuer
       ok = tc::mbar_wait(&bars->a_full, 0);
-      const uint32_t a_addr = tc::smem_u32(sA);
       for (int t = 0; ok && t < nB; ++t) {
-        const int s = t % kStages, u = t / kStages, b = t % kAcc, v = t / kAcc;
-        if (!tc::mbar_wait(&bars->acc_empty[b], (v & 1) ^ 1) ||
-            !tc::mbar_wait(&bars->full[s], u & 1)) {
+        const int s = t % kStages, u = t / kStages;
+        if (!tc::mbar_wait(&bars->full[s], u & 1)) {
           ok = false;
           break;
         }
-        tc::fence_after_sync();
         const uint32_t b_addr = tc::smem_u32(sB + s * TB);
+        for (int j = 0; j < kNA; ++j) {
+          if (!tc::mbar_wait(&bars->acc_empty[j], (t & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          tc::fence_after_sync();
+          const uint32_t a_addr = tc::smem_u32(sA + j * TA);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ks = (kk & 3) * 32;  // 16 bf16 = 32 bytes per K step
-          tc::mma_bf16(tmem + b * kBN, tc::desc_k_sw128(a_addr + (kk >> 2) * kHalfA + ks),
-                       tc::desc_k_sw128(b_addr + (kk >> 2) * kHalfB + ks), kIdesc,
-                       kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t ks = (kk & 3) * 32;  // 16 bf16 = 32 bytes per K step
+            tc::mma_bf16(tmem + j * kBN, tc::desc_k_sw128(a_addr + (kk >> 2) * kHalfA + ks),
+                         tc::desc_k_sw128(b_addr + (kk >> 2) * kHalfB + ks), kIdesc,
+                         kk > 0 ? 1u : 0u);
+          }
+          if (kPass == 2)  // + nl_q / c on every logit of query q
+            tc::mma_bf16(tmem + j * kBN, tc::desc_k_sw32(tc::smem_u32(sOnes)),
+                         tc::desc_k_sw32(tc::smem_u32(sX + s * kXBytes)), kIdesc, 1u);
+          tc::mma_commit(&bars->acc_full[j]);  // accumulator j ready
         }
-        if (kPass == 2)  // + nl_q / c on every logit of query q
-          tc::mma_bf16(tmem + b * kBN, tc::desc_k_sw32(tc::smem_u32(sOnes)),
-                       tc::desc_k_sw32(tc::smem_u32(sX + s * kXBytes)), kIdesc, 1u);
-        tc::mma_commit(&bars->empty[s]);     // operand stage reusable once read
-        tc::mma_commit(&bars->acc_full[b]);  // accumulator b ready
+        tc::mma_commit(&bars->empty[s]);  // operand stage reusable once both MMAs read it
       }
     }
-  } else if (warp >= 4) {  // ---- kEpi epilogue warpgroups, each on its column slice
-    const int g = (warp - 4) >> 2;
+  } else if (warp >= 4) {  // ---- epilogue: 4 kWG warpgroups per A tile, each on its column slice
+    const int e = warp - 4;
+    const int j = e / (4 * kWG);       // A tile (and accumulator) of this warp
+    const int g = (e / 4) % kWG;       // column slice within the tile
     const int sub = warp & 3;          // TMEM lane quarter
-    const int rloc = sub * 32 + lane;  // this thread's row of the A tile
-    const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16) + g * kSlice;
+    const int rloc = sub * 32 + lane;  // this thread's row of A tile j
+    const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16) + j * kBN + g * kSlice;
     float ref = -INFINITY, l = 0.0f;     // pass 1: reference and sum (log2 units)
     float2 acc = make_float2(0.f, 0.f);  // pass 2: column sum
     for (int t = 0; t < nB; ++t) {
-      const int b = t % kAcc, v = t / kAcc;
-      if (!tc::mbar_wait(&bars->acc_full[b], v & 1)) {
+      // the warp leaves together (the TMEM loads below are warp-collective)
+      if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->acc_full[j], t & 1))) {
         ok = false;
         break;
       }
       tc::fence_after_sync();
-      const uint32_t col0 = lane_addr + b * kBN;
       const int valid = Lk - (t_begin + t) * kBN - g * kSlice;  // pass 1: keys left
+      constexpr int kNch = kSlice / kCh;
+      if (kPass == 1 && valid >= kSlice) {
+        // A full slice: the chunks' overflow checks are folded into one flag,
+        // so no chunk but the last ends in a branch.  If a chunk before the
+        // last overflowed (rare), the slice is redone from TMEM, chunk by
+        // chunk with the exact check, before the accumulator is released.
+        const float l0 = l, ref0 = ref;
+        bool bad = false;
 #pragma unroll
-      for (int c = 0; c < kSlice / kCh; ++c) {
+        for (int c = 0; c < kNch; ++c) {
+          uint32_t ra[kCh];
+          // tcgen05.ld is warp-collective: the whole warp redoes the slice if
+          // any of its rows overflowed (the others recompute the same sums).
+          if (c + 1 == kNch && __any_sync(0xffffffffu, bad)) {
+            l = l0;
+            ref = ref0;
+            redo_chunks(lane_addr, kNch - 1, c2, ref, l);
+          }
+          tc::tmem_ld32(lane_addr + c * kCh, ra);
+          tc::tmem_ld_wait(ra);
+          if (c + 1 == kNch) {  // the slice is in registers: free the accumulator
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->acc_empty[j]);
+          }
+          if (c == 0 && ref == -INFINITY) ref = chunk_max(ra) * c2;
+          if (c + 1 < kNch) {
+            const float cs = chunk_sum_shifted(ra, c2, ref);
+            bad |= !(cs <= kRescaleAt);
+            l += cs;
+          } else {
+            row_chunk(ra, kCh, c2, ref, l);
+          }
+        }
+        continue;
+      }
+#pragma unroll
+      for (int c = 0; c < kNch; ++c) {
         uint32_t ra[kCh];
-        tc::tmem_ld32(col0 + c * kCh, ra);
+        tc::tmem_ld32(lane_addr + c * kCh, ra);
         tc::tmem_ld_wait(ra);
         if (c + 1 == kSlice / kCh) {  // the slice is in registers: free the accumulator
           tc::fence_before_sync();
           __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&bars->acc_empty[b]);
+          if (lane == 0) tc::mbar_arrive(&bars->acc_empty[j]);
         }
         if (kPass == 1)
           row_chunk(ra, valid - c * kCh, c2, ref, l);
@@ -357,24 +423,25 @@ __global__ void __launch_bounds__(kThreads, 1)
           col_chunk(ra, c2, acc);
       }
     }
-    // Merge the groups' partial results for each row (every group reaches
+    // Merge the slices' partial results for each row (every warp reaches
     // this barrier, also after a timeout).
+    float* mj = sM + (size_t)j * kWG * 2 * kBM;
     if (g > 0) {
-      sM[(2 * g) * kBM + rloc] = kPass == 1 ? ref : acc.x + acc.y;
-      sM[(2 * g + 1) * kBM + rloc] = l;
+      mj[(2 * g) * kBM + rloc] = kPass == 1 ? ref : acc.x + acc.y;
+      mj[(2 * g + 1) * kBM + rloc] = l;
     }
     epilogue_sync();
     if (g == 0 && ok) {
-      const int row = a0 + rloc;
+      const int row = a0 + j * kBM + rloc;
       if (kPass == 1) {
         float M = ref;
 #pragma unroll
-        for (int q = 1; q < kEpi; ++q) M = fmaxf(M, sM[(2 * q) * kBM + rloc]);
+        for (int q = 1; q < kWG; ++q) M = fmaxf(M, mj[(2 * q) * kBM + rloc]);
         float L = (ref == -INFINITY) ? 0.0f : l * tc::ex2(ref - M);
 #pragma unroll
-        for (int q = 1; q < kEpi; ++q) {
-          const float rq = sM[(2 * q) * kBM + rloc];
-          if (rq != -INFINITY) L += sM[(2 * q + 1) * kBM + rloc] * tc::ex2(rq - M);
+        for (int q = 1; q < kWG; ++q) {
+          const float rq = mj[(2 * q) * kBM + rloc];
+          if (rq != -INFINITY) L += mj[(2 * q + 1) * kBM + rloc] * tc::ex2(rq - M);
         }
         if (nsplit == 1)
           write_nlx(nlx + ((size_t)h * lq_pad + row) * 2, row < Lq ? -(M + __log2f(L)) : -INFINITY,
@@ -384,7 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         float sum = acc.x + acc.y;
 #pragma unroll
-        for (int q = 1; q < kEpi; ++q) sum += sM[(2 * q) * kBM + rloc];
+        for (int q = 1; q < kWG; ++q) sum += mj[(2 * q) * kBM + rloc];
         if (row < Lk) imp[(size_t)h * Lk + row] = sum / (float)Lq;
       }
     }
@@ -393,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
-  if (warp == 2) tc::tmem_dealloc(tmem, kAcc * kBN);
+  if (warp == 2) tc::tmem_dealloc(tmem, kNA * kBN);
 }
 
 // Combine the key-split partial (reference, sum) pairs of every query row.
@@ -506,7 +573,7 @@ cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, int ldk, fl
   e = cudaFuncSetAttribute(imp_tc_kernel<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
   if (e != cudaSuccess) return e;
-  const int nq = lq_pad / kBM;
+  const int nq = lq_pad / (kNA * kBM);
   const int nkt = (int)ceil_div(Lk, kBN);
   const int nsplit = choose_split(nq * H, nkt);
   imp_tc_kernel<D, 1><<<dim3(nq * nsplit, H), kThreads, smem, s>>>(
@@ -518,7 +585,7 @@ cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, int ldk, fl
     nl_merge_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(part, nsplit, H, Lq,
                                                                             lq_pad, c2, nlx);
   }
-  imp_tc_kernel<D, 2><<<dim3((unsigned)ceil_div(Lk, kBM), H), kThreads, smem, s>>>(
+  imp_tc_kernel<D, 2><<<dim3((unsigned)ceil_div(Lk, kNA * kBM), H), kThreads, smem, s>>>(
       mkA, mqB, mx, Lq, Lk, lq_pad, 1, c2, nlx, part, imp, err);
   return cudaGetLastError();
 }

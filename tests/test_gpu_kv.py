@@ -63,6 +63,32 @@ def test_importance_explicit_scale_and_sharp_softmax():
     _close(got, O.importance(f64(q), f64(k), scale=0.5), bf16=True)
 
 
+@pytest.mark.parametrize("d,dtype,grow", [(128, torch.bfloat16, 1), (64, torch.bfloat16, 1),
+                                           (128, torch.bfloat16, -1), (128, torch.float32, 1)])
+def test_importance_logits_drifting_along_keys(d, dtype, grow):
+    """Keys drift towards (grow=1) or away from (grow=-1) the queries' common
+    direction, so along a row the logits rise (or fall) by ~200 in log2 units
+    from the first key to the last, ~15 within every 128-key slice that one
+    epilogue warp drains: the row pass must move its reference again and
+    again, inside slices too (its rare overflow path), and the column pass
+    must still weigh every query by the right normaliser."""
+    g = torch.Generator().manual_seed(11 + d)
+    H, Lq, Lk = 2, 300, 1700
+    u = torch.randn(H, 1, d, generator=g)
+    u = u / u.norm(dim=-1, keepdim=True)
+    q = torch.randn(H, Lq, d, generator=g) * 0.3 + 3.0 * u
+    c = np.log2(np.e) / np.sqrt(d)
+    amp = 200.0 / (3.0 * c)  # q.k grows by ~3 * amp along the row
+    ramp = torch.linspace(0.0, 1.0, Lk) if grow > 0 else torch.linspace(1.0, 0.0, Lk)
+    k = torch.randn(H, Lk, d, generator=g) + (amp * ramp)[None, :, None] * u
+    q, k = q.to(dtype), k.to(dtype)
+    got = importance_gpu(q, k)
+    ref = O.importance(f64(q), f64(k))
+    assert np.all(np.isfinite(got))
+    _close(got, ref, bf16=dtype == torch.bfloat16)
+    np.testing.assert_allclose(got.sum(axis=1), 1.0, rtol=1e-4)
+
+
 @pytest.mark.parametrize("name", ["bf16_layer", "bf16_large_head"])
 def test_importance_workload_sampled_heads(name):
     """All heads go through the kernel; two heads are checked against the
