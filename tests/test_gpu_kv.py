@@ -50,7 +50,10 @@ def test_importance_tiny_fp32_full():
 @pytest.mark.parametrize("H,Lq,Lk,d,dtype", [
     (3, 300, 777, 128, torch.bfloat16), (2, 129, 1000, 64, torch.bfloat16),
     (1, 1, 5, 128, torch.bfloat16), (2, 257, 130, 64, torch.float32),
-    (1, 64, 64, 128, torch.float32), (2, 1000, 385, 128, torch.bfloat16)])
+    (1, 64, 64, 128, torch.float32), (2, 1000, 385, 128, torch.bfloat16),
+    # 306 key tiles of 128 (the last of each head partial): 148 two-tile CTAs
+    # and 10 one-tile CTAs in the column pass
+    (3, 300, 13000, 128, torch.bfloat16)])
 def test_importance_ragged(H, Lq, Lk, d, dtype):
     q, k = _rand_qk(H, Lq, Lk, d, dtype, seed=Lq + Lk)
     got = importance_gpu(q, k)
