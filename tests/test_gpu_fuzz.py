@@ -1,6 +1,7 @@
 """Seeded random cases for every call against the oracle: ragged sizes, both
 dtypes and head dims, random pooling windows, lambdas (also outside [0, 1]),
-budgets (also B >= L_k), explicit softmax scales, chunk counts and sizes that
+budgets (also B >= L_k), explicit softmax scales, cache commits of both dtypes
+(any chunk size, fewer candidates than the buffer holds), chunk counts and sizes that
 are not multiples of 4, inactive chunks and zero updates.  The tolerances and
 margin waivers are the ones the other parity tests use."""
 
@@ -173,3 +174,46 @@ def test_cache_commit_random(seed):
         assert torch.equal(kn[h, :B].cpu(), kb[h].index_select(0, sel))
         assert torch.equal(vn[h, :B].cpu(), vb[h].index_select(0, sel))
         assert torch.all(kn[h, B:] == 5.0)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_cache_commit_random_bf16(seed):
+    """The tensor-core path of a compression inside a cache buffer: random
+    head dims, chunk sizes that may not divide the budget, a clean count that
+    leaves fewer than B_budget + C candidates, the rows past them NaN."""
+    rng = np.random.default_rng(12000 + seed)
+    H = int(rng.integers(1, 4))
+    d = int(rng.choice([64, 128]))
+    C = int(rng.integers(100, 700))
+    B = int(rng.integers(C, 3 * C))
+    n = int(rng.integers(max(B - C + 1, 0), B + 1))
+    L = n + C
+    Lq = int(rng.integers(1, 400))
+    pool = int(rng.choice([1, 3, 7]))
+    lam = float(rng.uniform(0.2, 0.8))
+    g = torch.Generator().manual_seed(500 + seed)
+    kb = torch.full((H, B + C, d), float("nan")).to(torch.bfloat16)
+    vb = torch.full((H, B + C, d), float("nan")).to(torch.bfloat16)
+    kb[:, :L] = torch.randn(H, L, d, generator=g).to(torch.bfloat16)
+    vb[:, :L] = torch.randn(H, L, d, generator=g).to(torch.bfloat16)
+    q = torch.randn(H, Lq, d, generator=g).to(torch.bfloat16)
+    kn = torch.full_like(kb, 5.0).to(DEV)
+    vn = torch.full_like(vb, 5.0).to(DEV)
+    ws = fc.workspace(fc.fc_kv_cache_workspace_size(fc.FC_BF16, H, Lq, B, C, d))
+    idx = torch.empty(H, B, dtype=torch.int32, device=DEV)
+    n_next, comp = fc.fc_kv_cache_commit(q.to(DEV), kb.to(DEV), vb.to(DEV), kn, vn, n, C, ws,
+                                         pool, lam, idx=idx)
+    torch.cuda.synchronize()
+    assert comp and n_next == B
+    assert fc.fc_check_workspace(fc.FC_WS_CACHE, ws)
+    kc = f64(kb[:, :L])
+    sc_r = O.score(O.importance(f64(q), kc), O.redundancy(kc), lam, pool)
+    gi = idx.cpu().numpy()
+    assert gi.min() >= 0 and gi.max() < L
+    for h in range(H):
+        span = max(float(sc_r[h].max() - sc_r[h].min()), 1e-30)
+        assert_selection_matches(gi[h:h + 1], sc_r[h:h + 1].astype(np.float64), B, TOL_BF16 * span)
+        sel = torch.from_numpy(gi[h].astype(np.int64))
+        assert torch.equal(kn[h, :B].cpu(), kb[h].index_select(0, sel))
+        assert torch.equal(vn[h, :B].cpu(), vb[h].index_select(0, sel))
+        assert torch.all(kn[h, B:].float() == 5.0)
