@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(kCompactThreads)
     compact_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v, int Lk, int ldk, int B,
                    int ldo, const int32_t* __restrict__ idx, uint4* __restrict__ ko,
                    uint4* __restrict__ vo) {
+  grid_dep_wait();  // idx (and anything the kernel before touched) is ready
+  grid_dep_launch();
   constexpr int RPW = 32 / LPR;
   constexpr int kRowsPerStep = (kCompactThreads / 32) * RPW;
   constexpr int kRowsPerBlock = kRowsPerStep * kCompactUnroll;
@@ -58,9 +60,18 @@ cudaError_t run(const void* k, const void* v, int H, int Lk, int ldk, const int3
                 int ldo, void* ko, void* vo, cudaStream_t s) {
   constexpr int kRowsPerBlock = (kCompactThreads / 32) * (32 / LPR) * kCompactUnroll;
   dim3 grid((unsigned)ceil_div(B, kRowsPerBlock), H, 2);
-  compact_kernel<LPR><<<grid, kCompactThreads, 0, s>>>(
-      static_cast<const uint4*>(k), static_cast<const uint4*>(v), Lk, ldk, B, ldo, idx,
-      static_cast<uint4*>(ko), static_cast<uint4*>(vo));
+  // a programmatic dependent: scheduled while the selection finishes
+  cudaLaunchAttribute attr[1] = {pdl_attribute()};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kCompactThreads);
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(
+      &cfg, compact_kernel<LPR>, static_cast<const uint4*>(k), static_cast<const uint4*>(v), Lk,
+      ldk, B, ldo, idx, static_cast<uint4*>(ko), static_cast<uint4*>(vo));
+  if (e != cudaSuccess) return e;
   add_launches(1);
   return cudaGetLastError();
 }

@@ -37,6 +37,27 @@ template <> struct Vec16<__nv_bfloat16> {
   }
 };
 
+// Programmatic dependent launch.  grid_dep_wait: wait until the grid this
+// one programmatically depends on has completed and its memory is visible
+// (returns at once when the launch had no such dependency).  grid_dep_launch:
+// let the grid that depends on this one be scheduled now; it still waits
+// with grid_dep_wait before it touches anything this grid uses.
+__device__ __forceinline__ void grid_dep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_dep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Launch attribute that makes a kernel a programmatic dependent of the one
+// before it in the stream.
+inline cudaLaunchAttribute pdl_attribute() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
 // Streaming (read-once) 16-byte load that does not pollute L1.
 __device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
   uint4 r;

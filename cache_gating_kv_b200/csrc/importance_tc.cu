@@ -325,6 +325,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < KB; ++kb)
           tc::tma_load_3d(sA + j * TA + kb * kHalfA, &mapA, &bars->a_full, kb * 64,
                           a0 + j * kBM, h);
+      // Pass 2 may start while the row pass (or the merge) finishes: only the
+      // normaliser rows depend on it, so wait for it before the first stage.
+      if (kPass == 2) grid_dep_wait();
       for (int t = 0; t < nB; ++t) {
         const int s = t % kStages, u = t / kStages;
         if (!tc::mbar_wait(&bars->empty[s], (u & 1) ^ 1)) {
@@ -482,6 +485,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // Combine the key-split partial (reference, sum) pairs of every query row.
 __global__ void nl_merge_kernel(const float2* __restrict__ part, int nsplit, int H, int Lq,
                                 int lq_pad, float c2, uint4* __restrict__ nlx) {
+  grid_dep_wait();  // the row pass's partials
+  grid_dep_launch();
   const int64_t n = (int64_t)H * lq_pad;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -595,11 +600,25 @@ cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, int ldk, fl
   imp_tc_kernel<D, 1><<<dim3(nq * nsplit, H), kThreads, smem, s>>>(
       mqA, mkB, mx, Lq, Lk, lq_pad, nsplit, c2, nlx, part, imp, err, 0, 0);
   add_launches(nsplit > 1 ? 3 : 2);
+  // The merge and the column pass are launched as programmatic dependents of
+  // the kernel before them and wait for it (griddepcontrol.wait) only where
+  // they read what it wrote.  The passes themselves do not trigger their
+  // dependents early: column-pass CTAs waiting on idle SMs during the row
+  // pass's tail starved the redundancy kernel running beside the importance
+  // (measured: 27 us more per bench step).
+  cudaLaunchAttribute pdl[1] = {pdl_attribute()};
   if (nsplit > 1) {
     const int64_t n = (int64_t)H * lq_pad;
     const int64_t blocks = ceil_div(n, 256);
-    nl_merge_kernel<<<(unsigned)(blocks < 4096 ? blocks : 4096), 256, 0, s>>>(part, nsplit, H, Lq,
-                                                                            lq_pad, c2, nlx);
+    cudaLaunchConfig_t mc = {};
+    mc.gridDim = dim3((unsigned)(blocks < 4096 ? blocks : 4096));
+    mc.blockDim = dim3(256);
+    mc.stream = s;
+    mc.attrs = pdl;
+    mc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&mc, nl_merge_kernel, (const float2*)part, nsplit, H, Lq, lq_pad, c2,
+                           nlx);
+    if (e != cudaSuccess) return e;
   }
   // pass 2: whole waves of two-tile CTAs; a remainder of at most one wave's
   // worth of tiles goes to one-tile CTAs (half as long), else to pairs too
@@ -609,8 +628,16 @@ cudaError_t run(const void* q, const void* k, int H, int Lq, int Lk, int ldk, fl
   int64_t rem = tiles % wave2;
   if (rem > wave2 / 2) rem = 0;
   const int64_t npair = (tiles - rem) / 2;
-  imp_tc_kernel<D, 2><<<dim3((unsigned)(npair + rem), 1), kThreads, smem, s>>>(
-      mkA, mqB, mx, Lq, Lk, lq_pad, 1, c2, nlx, part, imp, err, tph, (int)npair);
+  cudaLaunchConfig_t pc = {};
+  pc.gridDim = dim3((unsigned)(npair + rem), 1);
+  pc.blockDim = dim3(kThreads);
+  pc.dynamicSmemBytes = smem;
+  pc.stream = s;
+  pc.attrs = pdl;
+  pc.numAttrs = 1;
+  e = cudaLaunchKernelEx(&pc, imp_tc_kernel<D, 2>, mkA, mqB, mx, Lq, Lk, lq_pad, 1, c2, nlx, part,
+                         imp, err, tph, (int)npair);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -213,6 +213,8 @@ __global__ void __launch_bounds__(kCsThreads)
     score_select_cluster_kernel(const float* __restrict__ imp, const float* __restrict__ red,
                                 int Lk, int r, float lam, float one_minus_lam, int B,
                                 float* __restrict__ score, int32_t* __restrict__ idx) {
+  grid_dep_wait();  // the kernel before this one (importance) has finished
+  grid_dep_launch();
   cg::cluster_group cluster = cg::this_cluster();
   const int nrank = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
@@ -417,13 +419,14 @@ cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk,
     cfg.blockDim = dim3(kCsThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)csize;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attribute();  // scheduled while the importance finishes
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = cudaLaunchKernelEx(&cfg, kern, imp, red, Lk, r, lambda, one_minus, B, score, idx);
     if (e != cudaSuccess) return e;
     add_launches(1);
