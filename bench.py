@@ -482,7 +482,7 @@ def native(a, rank, world, local_rank):
                      "flops_per_launch": exec_flops,
                      # DRAM read + write of the call's three launches, from the ncu capture
                      # of this kernel version (profiles/step_kernels_bf16_layer.md)
-                     "traffic": 267.3e6 if a.workload == "bf16_layer" else None,
+                     "traffic": 269.2e6 if a.workload == "bf16_layer" else None,
                      "traffic_unit": "bytes per call"},
         "kernels_ms": ms_call,
         "kernels_ms_alone": ms_alone,
