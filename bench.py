@@ -6,9 +6,11 @@ the libflowcache C-ABI:
   gate (fused Euler update + per-chunk relative L1 + accumulator) over every
   chunk, then importance, redundancy, pooled score + top-B, and K/V compaction
   over every head.
-Default workload: one bf16 layer (H=24, d=128, L_q=4096, L_k=16384, B=8192,
-lambda=0.5, pool 7) with the gate over 4 chunks of 24x45x45x16 fp32 latents
-(T=30, m=5, eps=0.01).
+Default workload: the long-history layer (H=40, d=128, L_q=8192, L_k=131072,
+B=32768, lambda=0.5, pool 7, bf16, 25% exact duplicate keys; no gate), the
+largest configuration that fits one GPU.  The same JSON line carries the full
+step of the full-step sweep at L_k=128K (40 layers of H=40, L_q=4096,
+B=32768, plus the 16-chunk gate over 24x45x45x16 fp32 latents).
 
 Metric: clean KV tokens scored+selected per second per head (= L_k / step
 time, summed over ranks); the gate's GB/s and each kernel's roofline fraction
@@ -19,7 +21,7 @@ ride along.  Multi-GPU (timing is the max over ranks, no data-path collective):
                             chunk is independent, so nothing is exchanged).
 
     python bench.py [--gpus N --steps K --warmup W] [--impl reference]
-                    [--workload NAME] [--shard layers|heads]
+                    [--workload NAME] [--shard layers|heads] [--heads N]
 """
 
 import argparse
@@ -63,15 +65,22 @@ def _args():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", default="bf16_layer")
+    ap.add_argument("--workload", default="long_history")
+    ap.add_argument("--heads", type=int, default=0,
+                    help="run only the first N heads of the layer (0 = all); for small "
+                         "profiler captures")
     ap.add_argument("--shard", default="layers", choices=["layers", "heads"])
     ap.add_argument("--serial", action="store_true",
                     help="run the five calls one after another on one stream")
-    ap.add_argument("--cpu-sample-heads", type=int, default=8)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-next", action="store_true",
                     help="skip the timings of the cache commit, mask consumer and history gate")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the full step of the full-step sweep (40 layers at L_k=128K)")
+    ap.add_argument("--ref-frac", type=int, default=16,
+                    help="the oracle legs time 1/N of a head's importance rows and a 1/N key "
+                         "subset of its redundancy per sampled head")
     return ap.parse_args()
 
 
@@ -212,18 +221,38 @@ def workload_desc(workload):
              if gate_cfg else "no gate"))
 
 
+def bench_config(workload, per_rank="one independent layer per GPU"):
+    """The ``config`` object of the JSON line; both arms report the same one."""
+    return {"workload": workload_desc(workload), "per_rank": per_rank,
+            "l2": "flushed between steps (256 MiB write + read-back, outside the timed events)"}
+
+
+# DRAM bytes (read + write) of one fc_kv_importance call, per head, from one
+# ncu capture of its launches (dram__bytes_read.sum + dram__bytes_write.sum) on
+# a subset of the workload's heads: workload -> (bytes per head, heads captured).
+# The traffic of the call grows in proportion to its heads (every head is an
+# independent slab of Q and K), so a full call is heads x the per-head bytes.
+# Keep in step with the kernel: a change to the importance kernels voids it.
+IMP_TRAFFIC_PER_HEAD = {}
+
+
+def _traffic(workload, H):
+    t = IMP_TRAFFIC_PER_HEAD.get(workload)
+    return None if t is None else t[0] * H
+
+
 class Step:
     """Device buffers of one step and the five C-ABI calls.  ``heads`` and
     ``chunks`` ([lo, hi) ranges) select this rank's share of the layer's heads
     and of the gate's chunks; by default the whole layer."""
 
-    def __init__(self, kv_cfg, gate_cfg, seed, dev, heads=None, chunks=None):
+    def __init__(self, kv_cfg, gate_cfg, seed, dev, heads=None, chunks=None, layer=0):
         import cache_gating_kv_b200 as fc
         from cache_gating_kv_b200 import workloads as W
 
         self.fc = fc
         self.kv, self.gc = kv_cfg, gate_cfg
-        q, k, v = W.kv_inputs(kv_cfg, seed=seed,
+        q, k, v = W.kv_inputs(kv_cfg, seed=seed, layer=layer,
                               heads=None if heads is None else range(*heads))
         self.host = {"q": q, "k": k, "v": v}
         n_c = 0
@@ -358,6 +387,9 @@ def native(a, rank, world, local_rank):
         step = Step(kv_cfg, gate_cfg, seed=0, dev=dev, heads=heads, chunks=chunks)
         per_rank = (f"heads [{heads[0]}, {heads[1]}) of one layer"
                     + (f", gate chunks [{chunks[0]}, {chunks[1]})" if chunks else ""))
+    elif a.heads > 0:
+        step = Step(kv_cfg, gate_cfg, seed=rank, dev=dev, heads=(0, min(a.heads, kv_cfg.H)))
+        per_rank = f"the first {min(a.heads, kv_cfg.H)} heads of one layer per GPU"
     else:
         step = Step(kv_cfg, gate_cfg, seed=rank, dev=dev)
         per_rank = "one independent layer per GPU"
@@ -435,6 +467,9 @@ def native(a, rank, world, local_rank):
         if not a.no_next:
             hbm0, tf0, _, _ = _peaks()
             nxt = _next_rows(step, dev, stream, flush, sink, max(3, min(a.steps, 10)), hbm0, tf0)
+        sweep = None
+        if not a.no_sweep:
+            sweep = _full_step_sweep(dev, stream, side, flush, sink, rank)
         barrier()
     del graph
     ms_step = sum(tot) / len(tot)
@@ -472,18 +507,15 @@ def native(a, rank, world, local_rank):
         "scaling": "strong" if by_heads else "weak",
         "vs_baseline": None, "dtype": kv_cfg.dtype if kv_cfg.dtype == "bf16" else "f32",
         "data": "synthetic (seeded AR(1) keys, N(0,1) queries/values, flow-matching toy latents)",
-        "config": {"workload": workload_desc(a.workload),
-                   "per_rank": per_rank,
-                   "l2": "flushed between steps (256 MiB write + read-back, outside the timed "
-                         "events)"},
+        "config": bench_config(a.workload, per_rank),
         "roofline": {"bound": "tensor", "kernel": "fc_kv_importance (2 passes)",
                      "achieved": imp_tf, "peak": tf_burst, "unit": "TFLOP/s",
                      "frac": imp_tf / tf_burst, "peak_source": f"{src} bf16 burst",
                      "flops_per_launch": exec_flops,
-                     # DRAM read + write of the call's three launches, from the ncu capture
-                     # of this kernel version (profiles/step_kernels_bf16_layer.md)
-                     "traffic": 269.2e6 if a.workload == "bf16_layer" else None,
-                     "traffic_unit": "bytes per call"},
+                     "frac_algorithmic": imp_tf / 2 / tf_burst,
+                     "traffic": _traffic(a.workload, H),
+                     "traffic_unit": "bytes per call (DRAM read + write of the call's "
+                                     "launches, from one ncu capture, scaled by heads)"},
         "kernels_ms": ms_call,
         "kernels_ms_alone": ms_alone,
         "kernels_note": "kernels_ms: spans inside the timed step (gate and redundancy share "
@@ -515,6 +547,8 @@ def native(a, rank, world, local_rank):
         "gpu_launches": launches,
         "clocks": ck,
     }
+    if sweep is not None:
+        out["full_step_sweep"] = sweep
     if e2e:
         out["e2e"] = {"value": layers * Lk / (e2e["ms"] * 1e-3), "unit": UNIT,
                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]}
@@ -608,19 +642,83 @@ def _next_rows(step, dev, stream, flush, sink, steps, hbm, tf_peak):
     }
 
 
-def _gate_alone(gc, seed, dev, stream, flush, sink, steps):
-    """Gate step over every chunk of ``gc`` alone, CUDA-graph timed (ms)."""
+def _full_step_sweep(dev, stream, side, flush, sink, seed, layers=40, steps=2, warm=1):
+    """The full step of the full-step sweep at L_k = 131072: ``layers`` layers
+    of H=40, L_q=4096, B=32768 through importance, redundancy, score/top-B and
+    compaction, plus one gate step over the 16 chunks, timed with CUDA events
+    on the launching stream (L2 flushed between steps).  The layers alternate
+    between two seeded layers' inputs (drawing 40 distinct layers on the host
+    would take minutes); each layer's K and V are 1.34 GB apiece, ten times the
+    L2, so no layer finds the previous one's data in cache."""
+    from cache_gating_kv_b200 import workloads as W
+
+    kv, gc = W.KV_CONFIGS["sweep_lk131072"], W.GATE_CONFIGS["full_step_sweep"]
+    import cache_gating_kv_b200 as fc
+
+    ls = [Step(kv, None, seed=seed, dev=dev, layer=i) for i in range(2)]
+    g = _gate_bufs(gc, seed, dev)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+
+    def one():
+        ev0.record(stream)
+        fork = torch.cuda.Event()
+        fork.record(stream)
+        s2 = side if side is not None else stream
+        s2.wait_event(fork)
+        fc.fc_chunk_l1_gate(g["x"], g["v"], g["dt"], g["st"], gc.m, gc.eps[0], g["f"], g["l1"],
+                            g["mask"], g["ws"], stream=s2)
+        for i in range(layers):
+            ls[i % 2].run(stream, side=side)
+        ev1.record(stream)
+
+    times = []
+    with torch.cuda.stream(stream):
+        for i in range(warm + steps):
+            flush_l2(flush, sink)
+            g["f"].zero_()
+            torch.cuda.synchronize()
+            one()
+            torch.cuda.synchronize()
+            if i >= warm:
+                times.append(ev0.elapsed_time(ev1))
+    ms = sum(times) / len(times)
+    H, Lq, Lk, d = kv.H, kv.Lq, kv.Lk, kv.d
+    del ls, g
+    return {"workload": f"{layers} layers x sweep_lk131072 (H={H} d={d} L_q={Lq} L_k={Lk} "
+                        f"B={kv.B} bf16) + gate {gc.n_chunks}x{gc.N} fp32",
+            "ms_per_step": ms, "steps": steps,
+            "tokens/s/head": layers * Lk / (ms * 1e-3),
+            "TFLOP/s importance-executed over the step": layers * 4.0 * H * Lq * Lk * d /
+            (ms * 1e-3) / 1e12,
+            "inputs": "two seeded layers' inputs, alternating over the 40 layers",
+            "timing": "CUDA events on the launching stream around the whole step (eager "
+                      "launches); the gate and each layer's redundancy on the side stream"}
+
+
+def _gate_bufs(gc, seed, dev):
+    """Device buffers of one gate step over every chunk of ``gc`` (every chunk
+    active, past its forced steps)."""
     import cache_gating_kv_b200 as fc
     from cache_gating_kv_b200 import workloads as W
 
-    x = torch.from_numpy(W.gate_initial(gc, seed)).to(dev)
-    v = torch.from_numpy(W.gate_velocity(gc, seed)).to(dev)
-    st = torch.full((gc.n_chunks,), gc.m + 3, dtype=torch.int32, device=dev)
-    dt = torch.full((gc.n_chunks,), 0.001, device=dev)
-    f = torch.zeros(gc.n_chunks, device=dev)
-    l1 = torch.zeros(gc.n_chunks, device=dev)
-    mask = torch.zeros(gc.n_chunks, dtype=torch.uint8, device=dev)
-    ws = fc.workspace(fc.fc_gate_workspace_size(gc.n_chunks, gc.N), dev)
+    n = gc.n_chunks
+    return {"x": torch.from_numpy(W.gate_initial(gc, seed)).to(dev),
+            "v": torch.from_numpy(W.gate_velocity(gc, seed)).to(dev),
+            "st": torch.full((n,), gc.m + 3, dtype=torch.int32, device=dev),
+            "dt": torch.full((n,), 0.001, device=dev), "f": torch.zeros(n, device=dev),
+            "l1": torch.zeros(n, device=dev),
+            "mask": torch.zeros(n, dtype=torch.uint8, device=dev),
+            "ws": fc.workspace(fc.fc_gate_workspace_size(n, gc.N), dev)}
+
+
+def _gate_alone(gc, seed, dev, stream, flush, sink, steps):
+    """Gate step over every chunk of ``gc`` alone, CUDA-graph timed (ms)."""
+    import cache_gating_kv_b200 as fc
+
+    b = _gate_bufs(gc, seed, dev)
+    x, v, st, dt, f, l1, mask, ws = (b[k] for k in ("x", "v", "st", "dt", "f", "l1", "mask",
+                                                    "ws"))
     e0 = torch.cuda.Event(enable_timing=True, external=True)
     e1 = torch.cuda.Event(enable_timing=True, external=True)
     fc.fc_chunk_l1_gate(x, v, dt, st, gc.m, gc.eps[0], f, l1, mask, ws, stream=stream)
@@ -696,14 +794,24 @@ def _e2e(step, stream, side, flush, sink, a, dev):
 # ---------------------------------------------------------------------------
 # CPU oracle legs
 # ---------------------------------------------------------------------------
-def _oracle_step_seconds(kv_cfg, gate_cfg, heads, seed=0):
-    """Oracle time for the compression of ``heads`` heads plus one full gate
-    step (0 when the workload has no gate)."""
+def _oracle_sample(kv_cfg, gate_cfg, head, frac, seed=0):
+    """Times the oracle, as it stands, on a bounded sample of one step and
+    returns ``(measured seconds, estimated seconds of the whole step)``.
+
+    The sample is one head of the layer: the importance over its first
+    L_q/frac query rows (every key; the rows are independent, so the head's
+    time is that x frac), the redundancy of its first L_k/frac keys (the
+    brute-force cosine matrix is L_k^2 work, so the head's time is estimated
+    as that x frac^2), the score/top-B and the compaction of the whole head, and
+    one full gate step (when the workload has one).  Step estimate = gate +
+    H x the head's estimate."""
     from cache_gating_kv_b200 import workloads as W
     from oracle import flowcache_oracle as O
 
-    q, k, v = W.kv_inputs(kv_cfg, seed=seed, heads=list(range(heads)))
-    q64 = q.float().numpy().astype(np.float64)
+    q, k, v = W.kv_inputs(kv_cfg, seed=seed, heads=[head % kv_cfg.H])
+    nq = max(1, kv_cfg.Lq // frac)
+    nr = max(2, kv_cfg.Lk // frac)
+    q64 = q[:, :nq].float().numpy().astype(np.float64)
     k64 = k.float().numpy().astype(np.float64)
     kf, vf = k.float().numpy(), v.float().numpy()
     lam = kv_cfg.lam[len(kv_cfg.lam) // 2]
@@ -719,10 +827,26 @@ def _oracle_step_seconds(kv_cfg, gate_cfg, heads, seed=0):
         t_gate = time.perf_counter() - t0
     t0 = time.perf_counter()
     imp = O.importance(q64, k64)
-    red = O.redundancy(k64)
-    _, idx = O.score_topb(imp, red, lam, kv_cfg.pool, kv_cfg.B)
+    t_imp = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    red = O.redundancy(k64[:, :nr])
+    t_red = time.perf_counter() - t0
+    red_full = np.resize(red, (1, kv_cfg.Lk))  # a full-length vector for the selection's timing
+    t0 = time.perf_counter()
+    _, idx = O.score_topb(imp, red_full, lam, kv_cfg.pool, kv_cfg.B)
     O.compact(kf, vf, idx)
-    return t_gate, (time.perf_counter() - t0) / heads
+    t_rest = time.perf_counter() - t0
+    measured = t_gate + t_imp + t_red + t_rest
+    head_est = t_imp * (kv_cfg.Lq / nq) + t_red * (kv_cfg.Lk / nr) ** 2 + t_rest
+    return measured, t_gate + kv_cfg.H * head_est
+
+
+def _sample_desc(kv_cfg, frac):
+    return (f"one head per sample: the importance of its first {max(1, kv_cfg.Lq // frac)} of "
+            f"{kv_cfg.Lq} query rows (x{frac}), the redundancy of its first "
+            f"{max(2, kv_cfg.Lk // frac)} of {kv_cfg.Lk} keys (x{frac}^2, quadratic work), the "
+            f"score/top-B and compaction of the whole head, plus one full gate step when the "
+            f"workload has one; step estimate = gate + H x head estimate")
 
 
 def _cores():
@@ -733,43 +857,45 @@ def _cores():
         return os.cpu_count()
 
 
-def cpu_baseline(a):
-    from cache_gating_kv_b200 import workloads as W
-
+def cpu_baseline(a, samples=4):
     kv_cfg, gate_cfg = configs(a.workload)
-    heads = max(1, min(a.cpu_sample_heads, kv_cfg.H))
-    t_gate, t_head = _oracle_step_seconds(kv_cfg, gate_cfg, heads)
-    t_step = t_gate + kv_cfg.H * t_head
+    est = [_oracle_sample(kv_cfg, gate_cfg, h, a.ref_frac)[1] for h in range(samples)]
+    t_step = sum(est) / len(est)
     return {"value": kv_cfg.Lk / t_step, "unit": UNIT, "cores": _cores(), "kind": "oracle",
-            "sample": f"{heads} of {kv_cfg.H} heads of the compression (importance, redundancy, "
-                      f"score/top-B, compaction) plus one full gate step; step time = gate + "
-                      f"H x per-head time"}
+            "sample": f"{samples} samples; " + _sample_desc(kv_cfg, a.ref_frac),
+            "est_ms_per_step": t_step * 1e3}
 
 
 def reference(a, rank):
+    """The reference arm: the oracle on the host cores, on this arm's workload,
+    metric and unit.  Each step times one bounded sample (`_oracle_sample`);
+    ``ms_per_step`` is the time measured per step, and the value is L_k over
+    the estimated time of a whole step."""
     if rank != 0:
         return None
-    from cache_gating_kv_b200 import workloads as W
-
     kv_cfg, gate_cfg = configs(a.workload)
-    times = []
+    meas, est = [], []
     for i in range(a.warmup + a.steps):
-        t_gate, t_head = _oracle_step_seconds(kv_cfg, gate_cfg, 1, seed=i)
+        m, e = _oracle_sample(kv_cfg, gate_cfg, i, a.ref_frac, seed=0)
         if i >= a.warmup:
-            times.append(t_gate + kv_cfg.H * t_head)
-    t = sum(times) / len(times)
-    value = kv_cfg.Lk / t
-    sample = ("each step: 1 of the layer's heads through the oracle's compression plus one "
-              "full gate step; step time = gate + H x per-head time")
+            meas.append(m)
+            est.append(e)
+    t_est = sum(est) / len(est)
+    value = kv_cfg.Lk / t_est
+    sample = _sample_desc(kv_cfg, a.ref_frac)
     return {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
-            "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup, "ms_per_step": t * 1e3,
+            "n_gpus": a.gpus, "steps": a.steps, "warmup": a.warmup,
+            "ms_per_step": sum(meas) / len(meas) * 1e3,
+            "est_ms_per_full_step": t_est * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic",
-            "config": {"workload": workload_desc(a.workload)},
+            "config": bench_config(a.workload),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": _cores(), "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
-                    "d2h_bytes_per_step": 0}}
+                    "d2h_bytes_per_step": 0},
+            "note": "ms_per_step is the time each step's sample took; value = L_k / "
+                    "est_ms_per_full_step, the sample scaled to a whole step"}
 
 
 def main():

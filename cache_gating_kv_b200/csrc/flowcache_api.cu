@@ -85,12 +85,19 @@ fc_status launched(cudaError_t e, const char* what) {
   return ok();
 }
 
-size_t elem_bytes(fc_dtype t) { return t == FC_BF16 ? 2 : 4; }
-
 bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
   const char* pa = static_cast<const char*>(a);
   const char* pb = static_cast<const char*>(b);
   return pa < pb + nb && pb < pa + na;
+}
+
+size_t elem_bytes(fc_dtype t) { return t == FC_BF16 ? 2 : 4; }
+
+// Two [n][N] float32 latent arrays, one written in place while the other is
+// read, must be disjoint (the kernel reads v through a non-aliasing pointer).
+bool latents_overlap(const float* x, const float* v, int n, int64_t N) {
+  const size_t bytes = (size_t)n * (size_t)N * sizeof(float);
+  return ranges_overlap(x, bytes, v, bytes);
 }
 
 fc_status check_kv_shape(fc_dtype dtype, int H, int L1, int L2, int d) {
@@ -155,6 +162,8 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
   if (n_per_chunk > 0) {  // empty chunks touch no latent memory
     FC_CHECK_PTR(x);
     FC_CHECK_PTR(v);
+    if (latents_overlap(x, v, n_chunks, n_per_chunk))
+      return fail(FC_ERR_INVALID_ARG, "x and v overlap (x is updated in place while v is read)");
   }
   FC_CHECK_PTR(dt);
   FC_CHECK_PTR(step);
@@ -182,6 +191,9 @@ fc_status fc_history_l1_gate(float* h_old, const float* h_new, int n_segments,
   if (n_per_segment > 0) {
     FC_CHECK_PTR(h_old);
     FC_CHECK_PTR(h_new);
+    if (latents_overlap(h_old, h_new, n_segments, n_per_segment))
+      return fail(FC_ERR_INVALID_ARG,
+                  "h_old and h_new overlap (h_old is overwritten while h_new is read)");
   }
   FC_CHECK_PTR(step);
   FC_CHECK_PTR(f);
@@ -209,6 +221,8 @@ fc_status fc_chunk_l1_gate_noalloc(float* x, const float* v, int n_chunks, int64
   if (n_per_chunk > 0) {
     FC_CHECK_PTR(x);
     FC_CHECK_PTR(v);
+    if (latents_overlap(x, v, n_chunks, n_per_chunk))
+      return fail(FC_ERR_INVALID_ARG, "x and v overlap (x is updated in place while v is read)");
   }
   FC_CHECK_PTR(dt);
   FC_CHECK_PTR(step);

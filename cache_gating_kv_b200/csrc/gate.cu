@@ -19,6 +19,10 @@
 // pair; the last block of a chunk to finish (an integer completion counter,
 // no spinning, no float atomics) sums the partials in a fixed order and runs
 // the recurrence, so the result is deterministic and one launch does it all.
+#include <cuda.h>
+
+#include <mutex>
+
 #include "fc_common.cuh"
 #include "fc_kernels.h"
 
@@ -253,10 +257,47 @@ constexpr size_t kGateNoAllocBytes =
 
 static __device__ __align__(256) unsigned char g_gate_scratch[kGateNoAllocBytes];
 
-// Device address of g_gate_scratch per device ordinal, filled on the first
-// call made with that device current.  In host code the array's name is only
-// a host-side stand-in, so the address must come from cudaGetSymbolAddress.
-void* g_gate_scratch_addr[128] = {nullptr};
+// Device address of g_gate_scratch per device ordinal, together with the id
+// of the context it was looked up in.  In host code the array's name is only
+// a host-side stand-in, so the address must come from cudaGetSymbolAddress,
+// made with that device current.  The first call on a device (and the first
+// after its primary context was destroyed, e.g. by cudaDeviceReset, which
+// gives the array a new address) looks it up; later calls reuse it.  A mutex
+// orders host threads that make their first call at the same time.
+struct ScratchAddr {
+  unsigned long long ctx_id;
+  void* addr;
+};
+constexpr int kMaxDevices = 128;
+ScratchAddr g_gate_scratch_addr[kMaxDevices] = {};
+std::mutex g_gate_scratch_mu;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id (for the life of the process) of the current context, or 0.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_cur == nullptr || get_id == nullptr || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 }  // namespace
 
 int gate_noalloc_max_chunks() { return kGateNoAllocMaxChunks; }
@@ -265,14 +306,21 @@ cudaError_t gate_noalloc_scratch(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
-  if (g_gate_scratch_addr[dev] == nullptr) {
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  // Before the runtime has made a context current the id is 0, and the
+  // address is looked up (which creates the primary context) on every call
+  // until it has.
+  const unsigned long long ctx = current_ctx_id();
+  std::lock_guard<std::mutex> lock(g_gate_scratch_mu);
+  ScratchAddr& s = g_gate_scratch_addr[dev];
+  if (s.addr == nullptr || ctx == 0 || s.ctx_id != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_gate_scratch);
     if (e != cudaSuccess) return e;
-    g_gate_scratch_addr[dev] = p;
+    s.addr = p;
+    s.ctx_id = ctx;
   }
-  *out = g_gate_scratch_addr[dev];
+  *out = s.addr;
   return cudaSuccess;
 }
 

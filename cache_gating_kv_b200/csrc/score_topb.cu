@@ -443,12 +443,14 @@ cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk,
   }
   const size_t staged = (size_t)kHistBytes + (size_t)Lk * 4;
   if (staged <= (size_t)kSelSmemLimit) {
-    cudaFuncSetAttribute(select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)staged);
+    const cudaError_t e = cudaFuncSetAttribute(
+        select_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)staged);
+    if (e != cudaSuccess) return e;
     select_kernel<true><<<H, kSelThreads, staged, s>>>(keys, Lk, B, idx);
   } else {
-    cudaFuncSetAttribute(select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         kHistBytes);
+    const cudaError_t e = cudaFuncSetAttribute(
+        select_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHistBytes);
+    if (e != cudaSuccess) return e;
     select_kernel<false><<<H, kSelThreads, kHistBytes, s>>>(keys, Lk, B, idx);
   }
   return cudaGetLastError();

@@ -134,9 +134,10 @@ size_t fc_gate_workspace_size(int n_chunks, int64_t n_per_chunk);
  *              word after the n_chunks counters) is reserved: this kernel
  *              has no device-side waits and never sets it.
  * x and v may be NULL when n_per_chunk == 0 (then L1_rel = 0 for every
- * active chunk).
+ * active chunk).  x and v must not overlap (x is written while v is read).
  * Errors: n_chunks < 1, n_per_chunk < 0, m < 0, null/host/misaligned
- * pointers -> FC_ERR_INVALID_ARG; small ws -> FC_ERR_WORKSPACE.
+ * pointers, overlapping x and v -> FC_ERR_INVALID_ARG; small ws ->
+ * FC_ERR_WORKSPACE.
  */
 fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per_chunk,
                            const float* dt, const int32_t* step, int32_t m, float eps,
@@ -158,7 +159,7 @@ fc_status fc_chunk_l1_gate(float* x, const float* v, int n_chunks, int64_t n_per
  * summed in float64, the recurrence runs in float32.
  *
  *   h_old     [n][N] float32, in/out: h_{t+1} in, h_t out (for active segments)
- *   h_new     [n][N] float32, h_t
+ *   h_new     [n][N] float32, h_t; must not overlap h_old
  *   step      [n] int32, steps since the segment started; < 0: inactive, untouched
  *   m, delta  forced refresh steps, threshold
  *   f         [n] float32, in/out window sum
@@ -191,7 +192,12 @@ fc_status fc_history_l1_gate(float* h_old, const float* h_new, int n_segments,
  *     memset on `stream`, then launches the gate kernel.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture.
+ *     before any stream capture.  The address is kept per device together
+ *     with the id of the context it belongs to; a call made after the
+ *     device's context was destroyed and created again (cudaDeviceReset)
+ *     looks it up again, so make the first call after a reset outside
+ *     stream capture too.  Host threads may make their first calls at the
+ *     same time: the lookup is serialised by a lock.
  *   - Every call shares the one array: calls whose work overlaps on the GPU
  *     (other streams, other host threads) race and give wrong results; order
  *     them on one stream or with events.

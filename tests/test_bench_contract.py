@@ -32,7 +32,8 @@ def test_reference_arm_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["value"] > 0 and d["higher_is_better"] is True
     assert d["metric"] == bench.METRIC and d["unit"] == bench.UNIT
-    assert d["config"]["workload"] == bench.workload_desc("tiny_fp32")
+    assert d["config"] == bench.bench_config("tiny_fp32")  # the native arm's config object
+    assert d["ms_per_step"] > 0 and d["est_ms_per_full_step"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
 
