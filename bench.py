@@ -78,6 +78,9 @@ def _args():
                     help="skip the timings of the cache commit, mask consumer and history gate")
     ap.add_argument("--no-sweep", action="store_true",
                     help="skip the full step of the full-step sweep (40 layers at L_k=128K)")
+    ap.add_argument("--sweep-lk", default="131072",
+                    help="comma-separated L_k values of the full-step sweep to time "
+                         "(of 4096, 16384, 65536, 131072)")
     ap.add_argument("--ref-frac", type=int, default=16,
                     help="the oracle legs time 1/N of a head's importance rows and a 1/N key "
                          "subset of its redundancy per sampled head")
@@ -461,15 +464,22 @@ def native(a, rank, world, local_rank):
                     for n, (e0, e1) in Step.SPANS.items():
                         alone[n].append(ev[e0].elapsed_time(ev[e1]))
             del g1
-        gate16 = _gate_alone(W.GATE_CONFIGS["full_step_sweep"], rank, dev, stream, flush, sink,
-                             a.steps)
+        gates = {}
+        for gname in ("bf16_layer", "bf16_large_head", "full_step_sweep"):
+            gc = W.GATE_CONFIGS[gname]
+            ms_g = _gate_alone(gc, rank, dev, stream, flush, sink, max(a.steps, 10))
+            gb = _bytes_gate(gc) / (ms_g * 1e-3) / 1e9
+            gates[gname] = {"chunks": gc.n_chunks, "n_per_chunk": gc.N, "us": ms_g * 1e3,
+                            "GB/s": gb, "frac_hbm": gb / _peaks()[0]}
         nxt = None
         if not a.no_next:
             hbm0, tf0, _, _ = _peaks()
             nxt = _next_rows(step, dev, stream, flush, sink, max(3, min(a.steps, 10)), hbm0, tf0)
         sweep = None
         if not a.no_sweep:
-            sweep = _full_step_sweep(dev, stream, side, flush, sink, rank)
+            sweep = {}
+            for lk in (int(x) for x in a.sweep_lk.split(",")):
+                sweep[f"L_k={lk}"] = _full_step_sweep(dev, stream, side, flush, sink, rank, lk)
         barrier()
     del graph
     ms_step = sum(tot) / len(tot)
@@ -523,11 +533,8 @@ def native(a, rank, world, local_rank):
                         "one after another on one stream, which the GB/s figures use",
         "gate": {"GB/s": gate_gbs, "frac_hbm": gate_gbs / hbm if gate_gbs else None},
         "next_rows": nxt,
-        "gate_full_step_sweep": {"chunks": 16, "us": gate16 * 1e3,
-                                 "GB/s": _bytes_gate(W.GATE_CONFIGS["full_step_sweep"]) /
-                                 (gate16 * 1e-3) / 1e9,
-                                 "frac_hbm": _bytes_gate(W.GATE_CONFIGS["full_step_sweep"]) /
-                                 (gate16 * 1e-3) / 1e9 / hbm},
+        "gate_workloads": dict(gates, note="each gate step alone, CUDA graph, L2 flushed "
+                               "before every replay; 12 B moved per latent element"),
         "timing": "one step captured as a CUDA graph, replayed per step; CUDA events are "
                   "graph nodes around each call" +
                   ("" if a.serial else "; gate and redundancy on a second, lower-priority "
@@ -642,17 +649,20 @@ def _next_rows(step, dev, stream, flush, sink, steps, hbm, tf_peak):
     }
 
 
-def _full_step_sweep(dev, stream, side, flush, sink, seed, layers=40, steps=2, warm=1):
-    """The full step of the full-step sweep at L_k = 131072: ``layers`` layers
-    of H=40, L_q=4096, B=32768 through importance, redundancy, score/top-B and
+def _full_step_sweep(dev, stream, side, flush, sink, seed, lk=131072, layers=40, steps=2,
+                     warm=1):
+    """The full step of the full-step sweep at one L_k: ``layers`` layers of
+    H=40, L_q=4096, B=L_k/4 through importance, redundancy, score/top-B and
     compaction, plus one gate step over the 16 chunks, timed with CUDA events
     on the launching stream (L2 flushed between steps).  The layers alternate
     between two seeded layers' inputs (drawing 40 distinct layers on the host
-    would take minutes); each layer's K and V are 1.34 GB apiece, ten times the
-    L2, so no layer finds the previous one's data in cache."""
+    would take minutes); at L_k = 131072 each layer's K and V are 1.34 GB
+    apiece, ten times the L2, so no layer finds the previous one's data in
+    cache (at L_k = 4096 a layer's K is 42 MB, and the alternation keeps the
+    two layers apart by one layer's traffic)."""
     from cache_gating_kv_b200 import workloads as W
 
-    kv, gc = W.KV_CONFIGS["sweep_lk131072"], W.GATE_CONFIGS["full_step_sweep"]
+    kv, gc = W.KV_CONFIGS[f"sweep_lk{lk}"], W.GATE_CONFIGS["full_step_sweep"]
     import cache_gating_kv_b200 as fc
 
     ls = [Step(kv, None, seed=seed, dev=dev, layer=i) for i in range(2)]
@@ -685,7 +695,7 @@ def _full_step_sweep(dev, stream, side, flush, sink, seed, layers=40, steps=2, w
     ms = sum(times) / len(times)
     H, Lq, Lk, d = kv.H, kv.Lq, kv.Lk, kv.d
     del ls, g
-    return {"workload": f"{layers} layers x sweep_lk131072 (H={H} d={d} L_q={Lq} L_k={Lk} "
+    return {"workload": f"{layers} layers x sweep_lk{lk} (H={H} d={d} L_q={Lq} L_k={Lk} "
                         f"B={kv.B} bf16) + gate {gc.n_chunks}x{gc.N} fp32",
             "ms_per_step": ms, "steps": steps,
             "tokens/s/head": layers * Lk / (ms * 1e-3),

@@ -30,12 +30,16 @@ namespace fc {
 
 namespace {
 constexpr int kGateThreads = 256;
-constexpr int kGateUnroll = 4;
+#ifndef FC_GATE_UNROLL
+#define FC_GATE_UNROLL 4
+#endif
+#ifndef FC_GATE_BLOCKS_PER_SM
+#define FC_GATE_BLOCKS_PER_SM 4
+#endif
+constexpr int kGateUnroll = FC_GATE_UNROLL;            // 16-byte vectors of x (and of v) in flight per thread
+constexpr int kGateBlocksPerSm = FC_GATE_BLOCKS_PER_SM;  // resident blocks per SM the grid is sized for
 constexpr int kGateMaxBlocksPerChunk = 1024;
 
-// kHist = false: the FlowCache gate (recompute resets f to 0).
-// kHist = true: the history-guided gate of the ARCache notes (关键设计 1,
-// HGC): a refresh step opens the next window, so f restarts at its own Delta.
 template <bool kHist>
 __device__ __forceinline__ void gate_finalize(int c, int st, int m, float eps, double num,
                                               double den, float* f, float* l1, uint8_t* mask) {
@@ -63,7 +67,26 @@ __device__ __forceinline__ void gate_finalize(int c, int st, int m, float eps, d
 
 // FlowCache: p = v*dt (rounded once), X <- X + p (rounded once).
 // History gate: p = h_t - h_{t+1} (rounded once), h_{t+1} <- h_t.
-// Both sum |p| and |X before the step| in float64.
+// |p| and |X before the step| of the four lanes of a vector are summed
+// pairwise in float32 (two roundings: relative error below 2^-23, as all
+// terms are non-negative), then widened and added to the float64 sums; the
+// per-element float64 conversions measured on the conversion unit otherwise.
+template <bool kHist>
+__device__ __forceinline__ void gate_vec(float4& x, const float4& v, float h, double& num,
+                                         double& den) {
+  const float p0 = kHist ? __fsub_rn(v.x, x.x) : __fmul_rn(v.x, h);
+  const float p1 = kHist ? __fsub_rn(v.y, x.y) : __fmul_rn(v.y, h);
+  const float p2 = kHist ? __fsub_rn(v.z, x.z) : __fmul_rn(v.z, h);
+  const float p3 = kHist ? __fsub_rn(v.w, x.w) : __fmul_rn(v.w, h);
+  num += (double)__fadd_rn(__fadd_rn(fabsf(p0), fabsf(p1)), __fadd_rn(fabsf(p2), fabsf(p3)));
+  den += (double)__fadd_rn(__fadd_rn(fabsf(x.x), fabsf(x.y)), __fadd_rn(fabsf(x.z), fabsf(x.w)));
+  x.x = kHist ? v.x : __fadd_rn(x.x, p0);
+  x.y = kHist ? v.y : __fadd_rn(x.y, p1);
+  x.z = kHist ? v.z : __fadd_rn(x.z, p2);
+  x.w = kHist ? v.w : __fadd_rn(x.w, p3);
+}
+
+// One element (the unaligned head and tail of a chunk), summed in float64.
 template <bool kHist>
 __device__ __forceinline__ void gate_elem(float& x, float vv, float h, double& num, double& den) {
   const float p = kHist ? __fsub_rn(vv, x) : __fmul_rn(vv, h);
@@ -73,7 +96,7 @@ __device__ __forceinline__ void gate_elem(float& x, float vv, float h, double& n
 }
 
 template <bool kHist>
-__global__ void __launch_bounds__(kGateThreads)
+__global__ void __launch_bounds__(kGateThreads, kGateBlocksPerSm)
     gate_kernel(float* __restrict__ x, const float* __restrict__ v, int64_t N,
                 const float* __restrict__ dt, const int32_t* __restrict__ step, int m, float eps,
                 float* __restrict__ f, float* __restrict__ l1, uint8_t* __restrict__ mask,
@@ -128,10 +151,7 @@ __global__ void __launch_bounds__(kGateThreads)
     for (int u = 0; u < kGateUnroll; ++u) {
       const int64_t i = base + (int64_t)u * kGateThreads;
       if (i < hi) {
-        gate_elem<kHist>(xa[u].x, va[u].x, h, num, den);
-        gate_elem<kHist>(xa[u].y, va[u].y, h, num, den);
-        gate_elem<kHist>(xa[u].z, va[u].z, h, num, den);
-        gate_elem<kHist>(xa[u].w, va[u].w, h, num, den);
+        gate_vec<kHist>(xa[u], va[u], h, num, den);
         __stcs(x4 + i, xa[u]);
       }
     }
@@ -187,11 +207,23 @@ __global__ void __launch_bounds__(kGateThreads)
   // Last block of chunk c: fixed-order sum of every block's partial.
   __threadfence();
   if (warp == 0) {
+    // Every lane sums partials lane, lane + 32, ... in that order; the loads
+    // of eight of them are issued before the first is added.
+    constexpr int kBatch = 8;
+    const double2* pc = partials + (size_t)c * kGateMaxBlocksPerChunk;
     double a = 0.0, d = 0.0;
-    for (int i = lane; i < bpc; i += 32) {
-      const double2 p = __ldcg(&partials[(size_t)c * kGateMaxBlocksPerChunk + i]);
-      a += p.x;
-      d += p.y;
+    for (int i0 = 0; i0 < bpc; i0 += 32 * kBatch) {
+      double2 p[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = i0 + u * 32 + lane;
+        p[u] = i < bpc ? __ldcg(pc + i) : make_double2(0.0, 0.0);
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        a += p[u].x;
+        d += p[u].y;
+      }
     }
     a = warp_sum(a);
     d = warp_sum(d);
@@ -220,8 +252,8 @@ cudaError_t launch_gate(float* x, const float* v, int n_chunks, int64_t N, const
   unsigned* counters = static_cast<unsigned*>(ws);
   double2* partials =
       reinterpret_cast<double2*>(static_cast<char*>(ws) + counters_bytes(n_chunks));
-  // Four resident 256-thread blocks per SM over the whole grid.
-  const int64_t target = (int64_t)sm_count() * 4;
+  // kGateBlocksPerSm resident 256-thread blocks per SM over the whole grid.
+  const int64_t target = (int64_t)sm_count() * kGateBlocksPerSm;
   int64_t bpc = ceil_div(target, n_chunks);
   const int64_t useful = ceil_div(N / 4 + 1, kGateThreads);  // >= one vector per thread
   if (bpc > useful) bpc = useful;

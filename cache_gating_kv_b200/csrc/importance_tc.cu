@@ -79,8 +79,13 @@ constexpr int kBM = 128;      // rows of the resident A tile (MMA M, TMEM lanes)
 constexpr int kBN = 256;      // rows of each streamed B tile (MMA N, TMEM columns)
 constexpr int kStages = 2;    // shared-memory ring depth (64 KB B tiles)
 constexpr int kNA = 2;        // A tiles per CTA, one TMEM accumulator of kBN columns each
-#ifndef FC_IMP_EMU_MASK
-#define FC_IMP_EMU_MASK 0x2222  // pairs 1, 5, 9, 13 of 16: 1/4 of the exponentials
+// Which of the 16 pairs of a 32-column chunk take the FMA-pipe exponential,
+// per pass (bit p: pair p).
+#ifndef FC_IMP_EMU_MASK1
+#define FC_IMP_EMU_MASK1 0x2222  // pairs 1, 5, 9, 13 of 16: 1/4 of the exponentials
+#endif
+#ifndef FC_IMP_EMU_MASK2
+#define FC_IMP_EMU_MASK2 0x2222
 #endif
 constexpr int kWG = 2;        // epilogue warpgroups per A tile; each owns kBN/kWG columns
 constexpr int kEpiWarps = kNA * kWG * 4;
@@ -96,9 +101,9 @@ constexpr size_t kLseOffset = 256;    // nl extra rows [H][Lq_pad][16] bf16, the
 constexpr int kMaxSplit = 4;          // pass 1 may split the key range in up to 4 parts
 constexpr float kRescaleAt = 4294967296.0f;  // 2^32
 
-// Which pairs of a 32-column chunk go to the FMA pipes (bit p of the mask).
+template <int kPass>
 __device__ __forceinline__ constexpr bool emulated_pair(int p) {
-  return ((FC_IMP_EMU_MASK >> p) & 1) != 0;
+  return (((kPass == 1 ? FC_IMP_EMU_MASK1 : FC_IMP_EMU_MASK2) >> p) & 1) != 0;
 }
 
 template <int D>
@@ -156,8 +161,9 @@ __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) {
   return make_float2(__uint_as_float(a), __uint_as_float(b));
 }
 
-__device__ __forceinline__ float2 exp2_pair(int p, float2 x, bool clamp_high) {
-  if (emulated_pair(p)) return clamp_high ? tc::ex2_poly2<true>(x) : tc::ex2_poly2<false>(x);
+template <int kPass>
+__device__ __forceinline__ float2 exp2_pair(int p, float2 x) {
+  if (emulated_pair<kPass>(p)) return tc::ex2_poly2<kPass == 1>(x);
   return make_float2(tc::ex2(x.x), tc::ex2(x.y));
 }
 
@@ -167,7 +173,7 @@ __device__ __forceinline__ float chunk_sum_shifted(const uint32_t (&r)[kCh], flo
   float2 a0 = make_float2(0.f, 0.f), a1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int p = 0; p < kCh / 2; ++p) {
-    const float2 e = exp2_pair(p, tc::ffma2(f2(r[2 * p], r[2 * p + 1]), cc, sh), true);
+    const float2 e = exp2_pair<1>(p, tc::ffma2(f2(r[2 * p], r[2 * p + 1]), cc, sh));
     if (p & 1)
       a1 = tc::fadd2(a1, e);
     else
@@ -229,7 +235,7 @@ __device__ __forceinline__ void col_chunk(const uint32_t (&r)[kCh], float c2, fl
   float2 a1 = make_float2(0.f, 0.f);
 #pragma unroll
   for (int p = 0; p < kCh / 2; ++p) {
-    const float2 e = exp2_pair(p, tc::ffma2(f2(r[2 * p], r[2 * p + 1]), cc, z), false);
+    const float2 e = exp2_pair<2>(p, tc::ffma2(f2(r[2 * p], r[2 * p + 1]), cc, z));
     if (p & 1)
       a1 = tc::fadd2(a1, e);
     else

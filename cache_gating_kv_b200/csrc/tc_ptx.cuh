@@ -199,16 +199,20 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // 2^x for a pair, on the FMA pipes instead of the special-function unit, so
 // that part of a tile's exponentials can run beside the MUFU ones.  Method:
 // Cody-Waite style range reduction x = n + f with n = round(x) (the
-// 1.5*2^23 rounding constant) and f in [-1/2, 1/2], a degree-5 polynomial for
-// 2^f whose coefficients we fitted (iteratively reweighted least squares for
-// relative error on Chebyshev nodes; cache_gating_kv_b200/csrc/gen_exp2_poly.py),
-// then n is added to the exponent field.  Max relative error 2.4e-7 for
-// x >= -125; inputs below -125 (including -inf) are clamped there, giving
-// about 2^-125 instead of 0.  With kClampHigh, inputs above 64 are clamped to
-// 64 (callers that must see overflow as a large value); without it the caller
-// guarantees x <= 126.
-template <bool kClampHigh>
+// 1.5*2^23 rounding constant) and f in [-1/2, 1/2], a polynomial for 2^f whose
+// coefficients we fitted (iteratively reweighted least squares for relative
+// error on Chebyshev nodes; cache_gating_kv_b200/csrc/gen_exp2_poly.py), then
+// n is added to the exponent field.  kDeg = 5: max relative error 2.4e-7;
+// kDeg = 4: 2.7e-6; kDeg = 3: 7.6e-5 (for x >= -125).  Inputs below -125
+// (including -inf) are clamped there, giving about 2^-125 instead of 0.  With
+// kClampHigh, inputs above 64 are clamped to 64 (callers that must see
+// overflow as a large value); without it the caller guarantees x <= 126.
+#ifndef FC_EXP_POLY_DEG
+#define FC_EXP_POLY_DEG 5
+#endif
+template <bool kClampHigh, int kDeg = FC_EXP_POLY_DEG>
 __device__ __forceinline__ float2 ex2_poly2(float2 x) {
+  static_assert(kDeg >= 3 && kDeg <= 5, "fitted degrees: 3, 4, 5");
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   x.x = fmaxf(x.x, -125.0f);
   x.y = fmaxf(x.y, -125.0f);
@@ -219,12 +223,26 @@ __device__ __forceinline__ float2 ex2_poly2(float2 x) {
   const float2 t = fadd2(x, make_float2(kRound, kRound));
   const float2 j = fadd2(t, make_float2(-kRound, -kRound));
   const float2 f = fadd2(x, make_float2(-j.x, -j.y));
-  float2 p = make_float2(1.3278164e-03f, 1.3278164e-03f);
-  p = ffma2(p, f, make_float2(9.6755559e-03f, 9.6755559e-03f));
-  p = ffma2(p, f, make_float2(5.5507079e-02f, 5.5507079e-02f));
-  p = ffma2(p, f, make_float2(2.4022119e-01f, 2.4022119e-01f));
-  p = ffma2(p, f, make_float2(6.9314694e-01f, 6.9314694e-01f));
-  p = ffma2(p, f, make_float2(1.0000001e+00f, 1.0000001e+00f));
+  float2 p;
+  if constexpr (kDeg == 5) {
+    p = make_float2(1.3278164e-03f, 1.3278164e-03f);
+    p = ffma2(p, f, make_float2(9.6755559e-03f, 9.6755559e-03f));
+    p = ffma2(p, f, make_float2(5.5507079e-02f, 5.5507079e-02f));
+    p = ffma2(p, f, make_float2(2.4022119e-01f, 2.4022119e-01f));
+    p = ffma2(p, f, make_float2(6.9314694e-01f, 6.9314694e-01f));
+    p = ffma2(p, f, make_float2(1.0000001e+00f, 1.0000001e+00f));
+  } else if constexpr (kDeg == 4) {
+    p = make_float2(9.5718065e-03f, 9.5718065e-03f);
+    p = ffma2(p, f, make_float2(5.5918004e-02f, 5.5918004e-02f));
+    p = ffma2(p, f, make_float2(2.4024703e-01f, 2.4024703e-01f));
+    p = ffma2(p, f, make_float2(6.9312179e-01f, 6.9312179e-01f));
+    p = ffma2(p, f, make_float2(9.9999928e-01f, 9.9999928e-01f));
+  } else {
+    p = make_float2(5.5186376e-02f, 5.5186376e-02f);
+    p = ffma2(p, f, make_float2(2.4261236e-01f, 2.4261236e-01f));
+    p = ffma2(p, f, make_float2(6.9325829e-01f, 6.9325829e-01f));
+    p = ffma2(p, f, make_float2(9.9992794e-01f, 9.9992794e-01f));
+  }
   // the low bits of t hold n (two's complement); n << 23 lands in the exponent
   const uint32_t ex = (__float_as_uint(t.x) << 23) + __float_as_uint(p.x);
   const uint32_t ey = (__float_as_uint(t.y) << 23) + __float_as_uint(p.y);
