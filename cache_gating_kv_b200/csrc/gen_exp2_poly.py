@@ -1,5 +1,5 @@
-"""Fit the degree-5 polynomial for 2^f, f in [-1/2, 1/2], used by ex2_poly2
-in tc_ptx.cuh (run: python gen_exp2_poly.py).
+"""Fit the polynomials for 2^f, f in [-1/2, 1/2], used by ex2_poly2 in
+tc_ptx.cuh (degrees 3, 4 and 5; run: python gen_exp2_poly.py).
 
 Iteratively reweighted least squares on 4000 Chebyshev nodes, minimising the
 relative error; prints the float32 coefficients (constant term first) and the
@@ -31,6 +31,7 @@ def max_rel_err_f32(c):
 
 
 if __name__ == "__main__":
-    c = fit()
-    print("coefficients (c0..c5):", [f"{v:.7e}" for v in c])
-    print("max relative error (float32 Horner):", max_rel_err_f32(c))
+    for deg in (3, 4, 5):
+        c = fit(deg)
+        print(f"degree {deg} coefficients (c0..c{deg}):", [f"{v:.7e}" for v in c])
+        print("  max relative error (float32 Horner):", max_rel_err_f32(c))

@@ -43,9 +43,12 @@
 //     warps has loaded its slice (measured 1-3 % faster than one A tile with
 //     two accumulators, and each B tile crosses from L2 once per 256 rows);
 //   - uses packed f32x2 FMA/ADD for the scale-and-shift and the running sums;
-//   - evaluates 1 of every 4 exponentials on the FMA pipes (ex2_poly2, a
-//     polynomial of our own) and the rest on the special-function unit (a
-//     sweep of the mix on B200 put the optimum there);
+//   - evaluates part of the exponentials on the FMA pipes (ex2_poly2, a
+//     degree-3 polynomial of our own: 1 in 4 in the row pass, 3 in 8 in the
+//     column pass) and the rest on the special-function unit (sweeps of the
+//     mix and the degree on B200 put the optimum there; the packed f16x2 and
+//     bf16x2 forms of ex2 retire no more exponentials per clock than the
+//     float32 one, 16 per SM);
 //   - in pass 1 shifts by a lagged reference instead of the exact running max:
 //     the reference only moves (with an exact rescale) when a chunk's sum
 //     exceeds 2^32, so the per-element max disappears from the common path;
@@ -80,12 +83,19 @@ constexpr int kBN = 256;      // rows of each streamed B tile (MMA N, TMEM colum
 constexpr int kStages = 2;    // shared-memory ring depth (64 KB B tiles)
 constexpr int kNA = 2;        // A tiles per CTA, one TMEM accumulator of kBN columns each
 // Which of the 16 pairs of a 32-column chunk take the FMA-pipe exponential,
-// per pass (bit p: pair p).
+// per pass (bit p: pair p), and the degree of its polynomial.  Measured on
+// B200 (both passes, three workloads): degree 3 with 1/4 of the row pass's
+// and 3/8 of the column pass's exponentials on the FMA pipes is 2-6 % faster
+// than degree 5 with 1/4 in both; masks whose register schedule spills
+// (e.g. 5 of 16 pairs) run 2-3x slower.
 #ifndef FC_IMP_EMU_MASK1
 #define FC_IMP_EMU_MASK1 0x2222  // pairs 1, 5, 9, 13 of 16: 1/4 of the exponentials
 #endif
 #ifndef FC_IMP_EMU_MASK2
-#define FC_IMP_EMU_MASK2 0x2222
+#define FC_IMP_EMU_MASK2 0x4A4A  // pairs 1, 3, 6, 9, 11, 14: 3/8
+#endif
+#ifndef FC_IMP_POLY_DEG
+#define FC_IMP_POLY_DEG 3  // relative error below 7.6e-5 per exponential
 #endif
 constexpr int kWG = 2;        // epilogue warpgroups per A tile; each owns kBN/kWG columns
 constexpr int kEpiWarps = kNA * kWG * 4;
@@ -163,7 +173,7 @@ __device__ __forceinline__ float2 f2(uint32_t a, uint32_t b) {
 
 template <int kPass>
 __device__ __forceinline__ float2 exp2_pair(int p, float2 x) {
-  if (emulated_pair<kPass>(p)) return tc::ex2_poly2<kPass == 1>(x);
+  if (emulated_pair<kPass>(p)) return tc::ex2_poly2<kPass == 1, FC_IMP_POLY_DEG>(x);
   return make_float2(tc::ex2(x.x), tc::ex2(x.y));
 }
 
@@ -654,7 +664,7 @@ __global__ void exp2_selftest_kernel(const float* x, float* y_mufu, float* y_pol
     const float2 v = make_float2(x[i], x[i + 1]);
     y_mufu[i] = tc::ex2(v.x);
     y_mufu[i + 1] = tc::ex2(v.y);
-    const float2 p = tc::ex2_poly2<false>(v);
+    const float2 p = tc::ex2_poly2<false, FC_IMP_POLY_DEG>(v);
     y_poly[i] = p.x;
     y_poly[i + 1] = p.y;
   }

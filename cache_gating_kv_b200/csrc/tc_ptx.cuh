@@ -207,10 +207,7 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 // (including -inf) are clamped there, giving about 2^-125 instead of 0.  With
 // kClampHigh, inputs above 64 are clamped to 64 (callers that must see
 // overflow as a large value); without it the caller guarantees x <= 126.
-#ifndef FC_EXP_POLY_DEG
-#define FC_EXP_POLY_DEG 5
-#endif
-template <bool kClampHigh, int kDeg = FC_EXP_POLY_DEG>
+template <bool kClampHigh, int kDeg>
 __device__ __forceinline__ float2 ex2_poly2(float2 x) {
   static_assert(kDeg >= 3 && kDeg <= 5, "fitted degrees: 3, 4, 5");
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23

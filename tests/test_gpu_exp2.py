@@ -1,7 +1,9 @@
 """Accuracy of the two exponentials the tensor-core importance kernel mixes,
 through the fc_selftest_exp2 C-ABI entry: the special-function unit
-(ex2.approx) and the FMA-pipe range reduction + degree-5 polynomial, against
-numpy's float64 exp2 (relative error bounds) and against each other."""
+(ex2.approx) and the FMA-pipe range reduction + degree-3 polynomial, against
+numpy's float64 exp2 (relative error bounds: 7.6e-5 for the polynomial, the
+maximum of its float32 evaluation over [-1/2, 1/2] that the fitting script
+prints; 2^-21 for the special-function unit) and against each other."""
 
 import ctypes
 
@@ -36,7 +38,7 @@ def test_polynomial_exp2_relative_error():
     ym, yp = _run(x)
     ref = np.exp2(x.astype(np.float64))
     rel_p = np.abs(yp - ref) / ref
-    assert rel_p.max() < 3e-7, rel_p.max()
+    assert rel_p.max() < 7.6e-5, rel_p.max()
     normal = x >= -126
     rel_m = np.abs(ym[normal] - ref[normal]) / ref[normal]
     assert rel_m.max() < 2.0 ** -21
@@ -47,7 +49,7 @@ def test_polynomial_exp2_clamps_below():
     x = np.array([-np.inf, -1e30, -200.0, -125.0], np.float32)
     ym, yp = _run(x)
     assert np.all(ym[:3] == 0)
-    np.testing.assert_allclose(yp, 2.0 ** -125, rtol=3e-7)
+    np.testing.assert_allclose(yp, 2.0 ** -125, rtol=7.6e-5)
 
 
 def test_bounded_wait_gives_up_and_context_stays_usable():
@@ -64,4 +66,4 @@ def test_bounded_wait_gives_up_and_context_stays_usable():
     assert int(err.item()) == 1
     # the device is still usable: a regular library call succeeds
     ym, yp = _run(np.array([0.0, 1.0], np.float32))
-    assert ym[1] == 2.0 and abs(yp[1] - 2.0) < 1e-6
+    assert ym[1] == 2.0 and abs(yp[1] - 2.0) < 2 * 7.6e-5
