@@ -44,7 +44,7 @@
 //     two accumulators, and each B tile crosses from L2 once per 256 rows);
 //   - uses packed f32x2 FMA/ADD for the scale-and-shift and the running sums;
 //   - evaluates part of the exponentials on the FMA pipes (ex2_poly2, a
-//     degree-3 polynomial of our own: 1 in 4 in the row pass, 3 in 8 in the
+//     degree-3 polynomial of our own: 3 in 16 in the row pass, 3 in 8 in the
 //     column pass) and the rest on the special-function unit (sweeps of the
 //     mix and the degree on B200 put the optimum there; the packed f16x2 and
 //     bf16x2 forms of ex2 retire no more exponentials per clock than the
@@ -84,12 +84,14 @@ constexpr int kStages = 2;    // shared-memory ring depth (64 KB B tiles)
 constexpr int kNA = 2;        // A tiles per CTA, one TMEM accumulator of kBN columns each
 // Which of the 16 pairs of a 32-column chunk take the FMA-pipe exponential,
 // per pass (bit p: pair p), and the degree of its polynomial.  Measured on
-// B200 (both passes, three workloads): degree 3 with 1/4 of the row pass's
-// and 3/8 of the column pass's exponentials on the FMA pipes is 2-6 % faster
-// than degree 5 with 1/4 in both; masks whose register schedule spills
-// (e.g. 5 of 16 pairs) run 2-3x slower.
+// B200 (both passes; one layer of 24 heads at L_k = 16384, 12 heads at
+// 131072, 40 heads at 32760): degree 3 with 3/16 of the row pass's and 3/8 of
+// the column pass's exponentials on the FMA pipes was the steadiest and,
+// under the power cap of the long heads, the fastest (5.90 ms against
+// 6.03-6.19 for degree 5 with 1/4 in both); masks whose register schedule
+// spills (5 or 8 of 16 pairs in some placements) run 2-3x slower.
 #ifndef FC_IMP_EMU_MASK1
-#define FC_IMP_EMU_MASK1 0x2222  // pairs 1, 5, 9, 13 of 16: 1/4 of the exponentials
+#define FC_IMP_EMU_MASK1 0x0222  // pairs 1, 5, 9 of 16: 3/16 of the exponentials
 #endif
 #ifndef FC_IMP_EMU_MASK2
 #define FC_IMP_EMU_MASK2 0x4A4A  // pairs 1, 3, 6, 9, 11, 14: 3/8
