@@ -236,7 +236,11 @@ def bench_config(workload, per_rank="one independent layer per GPU"):
 # The traffic of the call grows in proportion to its heads (every head is an
 # independent slab of Q and K), so a full call is heads x the per-head bytes.
 # Keep in step with the kernel: a change to the importance kernels voids it.
-IMP_TRAFFIC_PER_HEAD = {}
+IMP_TRAFFIC_PER_HEAD = {
+    # all 40 heads captured at once (the three metrics take one ncu pass):
+    # row pass 1662.2 + 12.9 MB, column pass 1438.9 + 20.4 MB
+    "long_history": (3134.4e6 / 40, 40),
+}
 
 
 def _traffic(workload, H):
@@ -523,6 +527,7 @@ def native(a, rank, world, local_rank):
                      "frac": imp_tf / tf_burst, "peak_source": f"{src} bf16 burst",
                      "flops_per_launch": exec_flops,
                      "frac_algorithmic": imp_tf / 2 / tf_burst,
+                     "frac_of_sustained_peak": imp_tf / tf_sus,
                      "traffic": _traffic(a.workload, H),
                      "traffic_unit": "bytes per call (DRAM read + write of the call's "
                                      "launches, from one ncu capture, scaled by heads)"},

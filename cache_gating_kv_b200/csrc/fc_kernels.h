@@ -50,7 +50,9 @@ cudaError_t launch_importance_simt(const void* q, const void* k, bool bf16, int 
                                    cudaStream_t s, int ldk = 0);
 
 // ---- redundancy ----------------------------------------------------------------
-size_t redundancy_ws_bytes(int H, int d);
+size_t redundancy_ws_bytes(int H, int Lk, int d);
+// Largest L_k the redundancy's fixed-point accumulators serve.
+int redundancy_max_lk();
 cudaError_t launch_redundancy(const void* k, bool bf16, int H, int Lk, int d, float* red,
                               void* ws, cudaStream_t s, int ldk = 0);
 

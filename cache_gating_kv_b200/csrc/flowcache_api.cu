@@ -126,7 +126,7 @@ CacheWs cache_ws(int H, int Lq, int B_budget, int C, int d) {
   w.idx = o;
   o = fc::align_up(o + (size_t)H * B_budget * sizeof(int32_t), 256);
   w.red_ws = o;
-  o = fc::align_up(o + fc::redundancy_ws_bytes(H, d), 256);
+  o = fc::align_up(o + fc::redundancy_ws_bytes(H, (int)cap, d), 256);
   w.score_ws = o;
   w.total = fc::align_up(o + fc::score_topb_ws_bytes(H, (int)cap), 256);
   return w;
@@ -353,7 +353,7 @@ fc_status fc_kv_importance(const void* q, const void* k, fc_dtype dtype, int H, 
 size_t fc_redundancy_workspace_size(fc_dtype dtype, int H, int Lk, int d) {
   (void)dtype;
   (void)Lk;
-  return (H < 1 || (d != 64 && d != 128)) ? 0 : fc::redundancy_ws_bytes(H, d);
+  return (H < 1 || Lk < 1 || (d != 64 && d != 128)) ? 0 : fc::redundancy_ws_bytes(H, Lk, d);
 }
 
 fc_status fc_kv_redundancy(const void* k, fc_dtype dtype, int H, int Lk, int d, float* red,
@@ -362,9 +362,11 @@ fc_status fc_kv_redundancy(const void* k, fc_dtype dtype, int H, int Lk, int d, 
   fc::g_launches = 0;
   fc_status st = check_kv_shape(dtype, H, Lk, Lk, d);
   if (st != FC_OK) return st;
-  if (ws == nullptr || ws_bytes < fc::redundancy_ws_bytes(H, d))
+  if (Lk > fc::redundancy_max_lk())
+    return fail(FC_ERR_UNSUPPORTED, "Lk must be <= %d (got %d)", fc::redundancy_max_lk(), Lk);
+  if (ws == nullptr || ws_bytes < fc::redundancy_ws_bytes(H, Lk, d))
     return fail(FC_ERR_WORKSPACE, "redundancy workspace needs %zu bytes",
-                fc::redundancy_ws_bytes(H, d));
+                fc::redundancy_ws_bytes(H, Lk, d));
   FC_CHECK_PTR(k);
   FC_CHECK_PTR(red);
   FC_CHECK_PTR(ws);
@@ -442,6 +444,8 @@ fc_status fc_kv_cache_commit(const void* q, const void* k_buf, const void* v_buf
   if (C < 1 || B_budget < C)
     return fail(FC_ERR_INVALID_ARG, "need 1 <= C <= B_budget (got C=%d, B_budget=%d)", C, B_budget);
   if ((int64_t)B_budget + C > INT32_MAX / 2) return fail(FC_ERR_INVALID_ARG, "B_budget + C too large");
+  if ((int64_t)B_budget + C > fc::redundancy_max_lk())
+    return fail(FC_ERR_UNSUPPORTED, "B_budget + C must be <= %d", fc::redundancy_max_lk());
   const int cap = B_budget + C;
   fc_status st = check_kv_shape(dtype, H, Lq, cap, d);
   if (st != FC_OK) return st;

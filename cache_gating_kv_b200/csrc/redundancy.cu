@@ -9,33 +9,47 @@
 // so the logits r_j need one reduction over K and one dot pass.  r_j lies in
 // [-1, 1], hence exp(r_j) cannot overflow and the softmax needs no max.
 //
-// One kernel, one thread-block cluster per head (8 or 16 CTAs, each owning a
-// contiguous slice of the head's rows):
-//   1. every CTA sums khat over its rows; the partial d-vectors are exchanged
-//      through distributed shared memory and every CTA adds them in rank order
-//      (identical s everywhere, deterministic);
-//   2. every CTA re-reads its rows backwards (the last ones read are still in
-//      L2), forms r_j and
-//      e_j = exp(r_j), writes e_j, and the per-CTA sums of e_j are exchanged
-//      the same way;
-//   3. every CTA scales its rows by 1/sum_j e_j.
-// The cluster barriers are hardware barriers (no spin loops).  Each lane
-// holds two 16-byte vectors of a row (16 bf16 or 8 fp32 elements), so a row's
-// reductions take log2(d*elem/32) shuffles; the per-row scalars use the
-// special-function unit (rsqrt, ex2: ~2^-22 relative error); every lane keeps
-// two or four rows' loads in flight.
-#include <cooperative_groups.h>
+// Three phases per head, each over fixed slices of its keys (one CTA per
+// slice; 512 or 1024 keys, by the head's size), so a head's result does not
+// depend on how many heads a call has:
+//   1. sum:       the slice's sum of khat, converted to 2^-32 fixed point and
+//                 added to the head's 64-bit integer accumulators (integer
+//                 addition is exact, so s is the same whatever order the
+//                 slices finish in);
+//   2. logits:    every row's r_j and e_j = exp(r_j) (written to red), and the
+//                 slice's sum of e_j added the same way;
+//   3. normalise: red_j *= 1 / sum_j e_j.
+// Phase 2 reads K a second time.  To serve that read from L2 instead of HBM,
+// the heads go in groups whose keys take at most 48 MB (80 MB for heads of
+// 8 MB and more), and launch g runs phase 1 of group g, phase 2 of group g-1
+// and phase 3 of group g-2: while one group's keys stream in from HBM for the
+// sum, the previous group's are re-read from L2 (two groups' keys, about the
+// 126 MB of L2 at most).  The
+// launches are programmatic dependents of each other: the sum CTAs of launch
+// g start as the SMs of launch g-1 free up; the logit and normalise CTAs wait
+// (griddepcontrol.wait) for launch g-1 to complete.  No CTA spins on another.
+#include <algorithm>
 
 #include "fc_common.cuh"
 #include "fc_kernels.h"
-
-namespace cg = cooperative_groups;
 
 namespace fc {
 
 namespace {
 constexpr int kRedThreads = 256;
 constexpr int kRedWarps = kRedThreads / 32;
+// Keys per CTA and the keys' bytes per head group.  Both depend on the head's
+// size only (its L_k, d and dtype), never on H, so a head's result does not
+// depend on the call.  Measured on B200 (bf16, d=128): heads of 4 MB (L_k =
+// 16384) ran best with 512-key slices in 48 MB groups (47 us for 24 heads
+// against 55-72 with 1024/2048-key slices or 80 MB groups); heads of 8 MB
+// and more with 1024-key slices in 80 MB groups (121 us for 40 heads of 32760
+// keys against 129; 414 us for 40 heads of 131072 against 471).
+constexpr int kSliceSmall = 512, kSliceLarge = 1024;
+constexpr size_t kGroupSmall = 48ull << 20, kGroupLarge = 80ull << 20;
+constexpr size_t kLargeHead = 8ull << 20;  // per-head key bytes from which the large shape is used
+constexpr double kFix = 4294967296.0;       // 2^32: scale of the fixed-point accumulators
+constexpr int kMaxLk = 1 << 26;             // keeps every accumulator below 2^63
 
 // Each lane holds two 16-byte vectors (32 contiguous bytes) of a row.
 template <typename T, int D>
@@ -85,178 +99,215 @@ __device__ __forceinline__ void unpack(const uint4 (&u)[2], float* e) {
   Vec16<T>::to_float(u[1], e + Vec16<T>::N);
 }
 
-// U: rows in flight per lane (two 16-byte loads each).
+__device__ __forceinline__ long long to_fix(double v) { return __double2ll_rn(v * kFix); }
+__device__ __forceinline__ double from_fix(long long v) { return (double)v * (1.0 / kFix); }
+
+// The phases of one launch, by CTA index: first n1*S CTAs sum heads
+// [h1, h1+n1), then n2*S CTAs form the logits of heads [h2, h2+n2), then n3*S
+// CTAs normalise heads [h3, h3+n3).
+struct Roles {
+  int h1, n1, h2, n2, h3, n3;
+};
+
+// Workspace: per head D fixed-point sums of khat, then per head the
+// fixed-point sum of e_j; zeroed at the start of every call.
+template <int D>
+__device__ __forceinline__ long long* s_fix(long long* ws, int h) {
+  return ws + (size_t)h * (D + 1);
+}
+
 template <typename T, int D, int U>
 __global__ void __launch_bounds__(kRedThreads)
-    red_cluster_kernel(const T* __restrict__ k, int Lk, int ldk, int h0, float* __restrict__ red) {
+    red_phase_kernel(const T* __restrict__ k, int Lk, int ldk, int rows, int S, Roles ro,
+                     long long* __restrict__ acc, float* __restrict__ red) {
+  // The next launch may start on the SMs this one frees; its phase-2 and
+  // phase-3 CTAs still wait for this whole launch.
+  grid_dep_launch();
   using L = RowLayout<T, D>;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int nrank = (int)cluster.num_blocks();
-  const int rank = (int)cluster.block_rank();
-  const int h = h0 + blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = lane / L::LPR, cl = lane % L::LPR;
-  const int per = (int)ceil_div(Lk, nrank);
-  const int lo = min(Lk, rank * per), hi = min(Lk, lo + per);
-  const T* kh = k + (size_t)h * ldk * D;
   constexpr int kRowsPerIter = kRedWarps * L::RPW * U;
+  const int b = blockIdx.x;
+  int phase, h, sl;
+  if (b < ro.n1 * S) {
+    phase = 1;
+    h = ro.h1 + b / S;
+    sl = b % S;
+  } else if (b < (ro.n1 + ro.n2) * S) {
+    const int c = b - ro.n1 * S;
+    phase = 2;
+    h = ro.h2 + c / S;
+    sl = c % S;
+  } else {
+    const int c = b - (ro.n1 + ro.n2) * S;
+    phase = 3;
+    h = ro.h3 + c / S;
+    sl = c % S;
+  }
+  const int lo = sl * rows, hi = min(Lk, lo + rows);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int sub = lane / L::LPR, cl = lane % L::LPR;
+  const T* kh = k + (size_t)h * ldk * D;
+  long long* sh = s_fix<D>(acc, h);  // [D] sums of khat, then [1] sum of e
+  float* rh = red + (size_t)h * Lk;
 
   __shared__ float s_acc[kRedWarps][D];
-  __shared__ float s_part[D];  // this CTA's sum of khat (read by the whole cluster)
-  __shared__ float s_vec[D];   // the head's s
+  __shared__ float s_vec[D];
   __shared__ double s_esum[kRedWarps];
-  __shared__ double s_epart;   // this CTA's sum of e (read by the whole cluster)
-  __shared__ float s_inv;
 
-  // ---- 1. sum of the normalised rows --------------------------------------
-  float acc[L::EPL];
+  if (phase == 1) {  // ---- sum of the slice's normalised rows ----------------
+    float a[L::EPL];
 #pragma unroll
-  for (int i = 0; i < L::EPL; ++i) acc[i] = 0.0f;
-  for (int r0 = lo + warp * L::RPW * U; r0 < hi; r0 += kRowsPerIter) {
-    uint4 raw[U][2];
-    load_rows<T, D, U>(kh, r0, hi, sub, cl, raw);
+    for (int i = 0; i < L::EPL; ++i) a[i] = 0.0f;
+    for (int r0 = lo + warp * L::RPW * U; r0 < hi; r0 += kRowsPerIter) {
+      uint4 raw[U][2];
+      load_rows<T, D, U>(kh, r0, hi, sub, cl, raw);
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      float e[L::EPL];
-      unpack<T, D>(raw[u], e);
-      float n2 = 0.0f;
+      for (int u = 0; u < U; ++u) {
+        float e[L::EPL];
+        unpack<T, D>(raw[u], e);
+        float n2 = 0.0f;
 #pragma unroll
-      for (int i = 0; i < L::EPL; ++i) n2 = fmaf(e[i], e[i], n2);
-      n2 = row_sum<L::LPR>(n2);
-      const float inv = inv_norm(n2);  // a zero key stays zero
+        for (int i = 0; i < L::EPL; ++i) n2 = fmaf(e[i], e[i], n2);
+        n2 = row_sum<L::LPR>(n2);
+        const float inv = inv_norm(n2);  // a zero key (or a row past hi) adds zero
 #pragma unroll
-      for (int i = 0; i < L::EPL; ++i) acc[i] = fmaf(e[i], inv, acc[i]);
-    }
-  }
-#pragma unroll
-  for (int o = L::LPR; o < 32; o <<= 1)
-#pragma unroll
-    for (int i = 0; i < L::EPL; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
-  if (sub == 0) {
-#pragma unroll
-    for (int i = 0; i < L::EPL; ++i) s_acc[warp][cl * L::EPL + i] = acc[i];
-  }
-  __syncthreads();
-  for (int c = threadIdx.x; c < D; c += kRedThreads) {
-    float t = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kRedWarps; ++w) t += s_acc[w][c];
-    s_part[c] = t;
-  }
-  cluster.sync();
-  for (int c = threadIdx.x; c < D; c += kRedThreads) {
-    double t = 0.0;
-    for (int q = 0; q < nrank; ++q) t += (double)*cluster.map_shared_rank(&s_part[c], q);
-    s_vec[c] = (float)t;
-  }
-  __syncthreads();
-
-  // ---- 2. logits r_j and e_j = exp(r_j) -------------------------------------
-  float sv[L::EPL];
-#pragma unroll
-  for (int i = 0; i < L::EPL; ++i) sv[i] = s_vec[cl * L::EPL + i];
-  const float inv_lk = 1.0f / (float)Lk;
-  float* rh = red + (size_t)h * Lk;
-  double esum = 0.0;
-  // Backwards over the slice: the rows read last by step 1 come first, while
-  // they are still in L2.
-  const int n_iter = (int)ceil_div(hi - lo, kRowsPerIter);
-  for (int it = n_iter - 1; it >= 0; --it) {
-    const int r0 = lo + it * kRowsPerIter + warp * L::RPW * U;
-    uint4 raw[U][2];
-    load_rows<T, D, U>(kh, r0, hi, sub, cl, raw);
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
-      float e[L::EPL];
-      unpack<T, D>(raw[u], e);
-      float n2 = 0.0f, dot = 0.0f;
-#pragma unroll
-      for (int i = 0; i < L::EPL; ++i) {
-        n2 = fmaf(e[i], e[i], n2);
-        dot = fmaf(e[i], sv[i], dot);
-      }
-      n2 = row_sum<L::LPR>(n2);
-      dot = row_sum<L::LPR>(dot);
-      const float inv = inv_norm(n2);
-      // r_j = (khat_j . s - ||khat_j||^2) / L_k
-      const float rj = (dot * inv - n2 * inv * inv) * inv_lk;
-      const float ej = exp_fast(rj);
-      const int r = r0 + u * L::RPW + sub;
-      if (r < hi && cl == 0) {
-        rh[r] = ej;
-        esum += (double)ej;
+        for (int i = 0; i < L::EPL; ++i) a[i] = fmaf(e[i], inv, a[i]);
       }
     }
-  }
-  esum = warp_sum(esum);
-  if (lane == 0) s_esum[warp] = esum;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    double t = 0.0;
 #pragma unroll
-    for (int w = 0; w < kRedWarps; ++w) t += s_esum[w];
-    s_epart = t;
+    for (int o = L::LPR; o < 32; o <<= 1)
+#pragma unroll
+      for (int i = 0; i < L::EPL; ++i) a[i] += __shfl_xor_sync(0xffffffffu, a[i], o);
+    if (sub == 0) {
+#pragma unroll
+      for (int i = 0; i < L::EPL; ++i) s_acc[warp][cl * L::EPL + i] = a[i];
+    }
+    __syncthreads();
+    for (int c = tid; c < D; c += kRedThreads) {
+      float t = 0.0f;
+#pragma unroll
+      for (int w = 0; w < kRedWarps; ++w) t += s_acc[w][c];
+      atomicAdd(reinterpret_cast<unsigned long long*>(sh + c), (unsigned long long)to_fix(t));
+    }
+    return;
   }
-  cluster.sync();
-  if (threadIdx.x == 0) {
-    double z = 0.0;
-    for (int q = 0; q < nrank; ++q) z += *cluster.map_shared_rank(&s_epart, q);
-    s_inv = (float)(1.0 / z);
-  }
-  cluster.sync();  // no CTA leaves while another may still read its shared memory
 
-  // ---- 3. normalise this CTA's rows ----------------------------------------------
-  const float inv = s_inv;
-  for (int r = lo + threadIdx.x; r < hi; r += kRedThreads) rh[r] = rh[r] * inv;
+  grid_dep_wait();  // the sums (phase 2) or the e_j (phase 3) of the launch before
+  if (phase == 2) {  // ---- logits r_j and e_j = exp(r_j) ---------------------
+    for (int c = tid; c < D; c += kRedThreads) s_vec[c] = (float)from_fix(__ldcg(sh + c));
+    __syncthreads();
+    float sv[L::EPL];
+#pragma unroll
+    for (int i = 0; i < L::EPL; ++i) sv[i] = s_vec[cl * L::EPL + i];
+    const float inv_lk = 1.0f / (float)Lk;
+    double esum = 0.0;
+    for (int r0 = lo + warp * L::RPW * U; r0 < hi; r0 += kRowsPerIter) {
+      uint4 raw[U][2];
+      load_rows<T, D, U>(kh, r0, hi, sub, cl, raw);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float e[L::EPL];
+        unpack<T, D>(raw[u], e);
+        float n2 = 0.0f, dot = 0.0f;
+#pragma unroll
+        for (int i = 0; i < L::EPL; ++i) {
+          n2 = fmaf(e[i], e[i], n2);
+          dot = fmaf(e[i], sv[i], dot);
+        }
+        n2 = row_sum<L::LPR>(n2);
+        dot = row_sum<L::LPR>(dot);
+        const float inv = inv_norm(n2);
+        // r_j = (khat_j . s - ||khat_j||^2) / L_k
+        const float rj = (dot * inv - n2 * inv * inv) * inv_lk;
+        const float ej = exp_fast(rj);
+        const int r = r0 + u * L::RPW + sub;
+        if (r < hi && cl == 0) {
+          rh[r] = ej;
+          esum += (double)ej;
+        }
+      }
+    }
+    esum = warp_sum(esum);
+    if (lane == 0) s_esum[warp] = esum;
+    __syncthreads();
+    if (tid == 0) {
+      double t = 0.0;
+#pragma unroll
+      for (int w = 0; w < kRedWarps; ++w) t += s_esum[w];
+      atomicAdd(reinterpret_cast<unsigned long long*>(sh + D), (unsigned long long)to_fix(t));
+    }
+    return;
+  }
+
+  // ---- phase 3: normalise the slice ---------------------------------------------
+  const float inv = (float)(1.0 / from_fix(__ldcg(sh + D)));
+  for (int r = lo + tid; r < hi; r += kRedThreads) rh[r] = rh[r] * inv;
 }
 
 template <typename T, int D>
-cudaError_t run(const T* k, int H, int Lk, int ldk, float* red, cudaStream_t s) {
-  // 16 CTAs per head when the slices stay long enough, else the portable 8.
-  const int csize = (Lk >= 16 * 64) ? 16 : 8;
-  // Long heads keep four rows per lane in flight (two measured 17 % slower at
-  // L_k = 131072); short ones two (four measured 17 % slower at 16384).
-  auto kern = Lk >= 65536 ? red_cluster_kernel<T, D, 4> : red_cluster_kernel<T, D, 2>;
-  if (csize > 8) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    if (e != cudaSuccess) return e;
-  }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)csize, (unsigned)H, 1);
-  cfg.blockDim = dim3(kRedThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = (unsigned)csize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, k, Lk, ldk, 0, red);
+cudaError_t run(const T* k, int H, int Lk, int ldk, float* red, void* ws, cudaStream_t s) {
+  constexpr int U = 4;  // rows in flight per lane (two 16-byte loads each)
+  auto kern = red_phase_kernel<T, D, U>;
+  const size_t head_bytes = (size_t)Lk * D * sizeof(T);
+  const bool large = head_bytes >= kLargeHead;
+  const int rows = large ? kSliceLarge : kSliceSmall;
+  const size_t group_bytes = large ? kGroupLarge : kGroupSmall;
+  const int S = (int)ceil_div(Lk, rows);
+  const int G = (int)std::max<size_t>(1, std::min<size_t>(H, group_bytes / head_bytes));
+  const int nG = (int)ceil_div(H, G);
+  long long* acc = static_cast<long long*>(ws);
+  cudaError_t e = cudaMemsetAsync(acc, 0, (size_t)H * (D + 1) * sizeof(long long), s);
   if (e != cudaSuccess) return e;
   add_launches(1);
+  cudaLaunchAttribute pdl[1] = {pdl_attribute()};
+  auto heads = [&](int g, int& h0, int& n) {
+    if (g < 0 || g >= nG) {
+      h0 = 0;
+      n = 0;
+      return;
+    }
+    h0 = g * G;
+    n = std::min(G, H - h0);
+  };
+  for (int g = 0; g < nG + 2; ++g) {
+    Roles ro;
+    heads(g, ro.h1, ro.n1);
+    heads(g - 1, ro.h2, ro.n2);
+    heads(g - 2, ro.h3, ro.n3);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((ro.n1 + ro.n2 + ro.n3) * S));
+    cfg.blockDim = dim3(kRedThreads);
+    cfg.stream = s;
+    // The first launch follows the memset (and whatever wrote K) in plain
+    // stream order; the later ones are programmatic dependents.
+    cfg.attrs = g > 0 ? pdl : nullptr;
+    cfg.numAttrs = g > 0 ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, k, Lk, ldk, rows, S, ro, acc, red);
+    if (e != cudaSuccess) return e;
+    add_launches(1);
+  }
   return cudaSuccess;
 }
 }  // namespace
 
-size_t redundancy_ws_bytes(int H, int d) {
-  (void)H;
-  (void)d;
-  return 256;  // the fused kernel keeps its partial sums in (distributed) shared memory
+size_t redundancy_ws_bytes(int H, int Lk, int d) {
+  (void)Lk;
+  return align_up((size_t)H * (d + 1) * sizeof(long long), 256);
 }
+
+int redundancy_max_lk() { return kMaxLk; }
 
 cudaError_t launch_redundancy(const void* k, bool bf16, int H, int Lk, int d, float* red,
                               void* ws, cudaStream_t s, int ldk) {
-  (void)ws;
   if (ldk <= 0) ldk = Lk;
+  if (Lk > kMaxLk) return cudaErrorInvalidValue;
   if (bf16) {
     const __nv_bfloat16* kb = static_cast<const __nv_bfloat16*>(k);
-    return d == 128 ? run<__nv_bfloat16, 128>(kb, H, Lk, ldk, red, s)
-                    : run<__nv_bfloat16, 64>(kb, H, Lk, ldk, red, s);
+    return d == 128 ? run<__nv_bfloat16, 128>(kb, H, Lk, ldk, red, ws, s)
+                    : run<__nv_bfloat16, 64>(kb, H, Lk, ldk, red, ws, s);
   }
   const float* kf = static_cast<const float*>(k);
-  return d == 128 ? run<float, 128>(kf, H, Lk, ldk, red, s) : run<float, 64>(kf, H, Lk, ldk, red, s);
+  return d == 128 ? run<float, 128>(kf, H, Lk, ldk, red, ws, s)
+                  : run<float, 64>(kf, H, Lk, ldk, red, ws, s);
 }
 
 }  // namespace fc

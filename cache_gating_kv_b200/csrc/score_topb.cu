@@ -208,6 +208,7 @@ constexpr int kCsThreads = 512;  // 256 measured 8 % (L_k 16384) to 27 % (131072
 constexpr int kCsWarps = kCsThreads / 32;
 static_assert(kCsThreads >= 256, "one thread per histogram bin");
 constexpr int kCsMaxSlice = 12288;  // keys per CTA held in shared memory
+constexpr int kCsMaxCluster = 16;   // CTAs per cluster (one head)
 
 __global__ void __launch_bounds__(kCsThreads)
     score_select_cluster_kernel(const float* __restrict__ imp, const float* __restrict__ red,
@@ -236,19 +237,44 @@ __global__ void __launch_bounds__(kCsThreads)
   __shared__ int s_wgt[kCsWarps], s_wtie[kCsWarps];
 
   // ---- scores of the slice -> order-preserving keys ------------------------
+  // Imp and Red were just written by the kernels before: each thread issues
+  // kLd loads before it uses the first, so their L2 latencies overlap.
+  constexpr int kLd = 8;
   const float* ih = imp + (size_t)h * Lk;
   const float* rh = red + (size_t)h * Lk;
-  for (int t = tid; t < n + 2 * r; t += kCsThreads) {
-    const int j = lo - r + t;
-    tile[t] = (j >= 0 && j < Lk) ? ih[j] : -INFINITY;  // out-of-range taps ignored
+  const int nt = n + 2 * r;
+  for (int t0 = tid; t0 < nt; t0 += kCsThreads * kLd) {
+    float v[kLd];
+#pragma unroll
+    for (int u = 0; u < kLd; ++u) {
+      const int t = t0 + u * kCsThreads, j = lo - r + t;
+      v[u] = (t < nt && j >= 0 && j < Lk) ? ih[j] : -INFINITY;  // out-of-range taps ignored
+    }
+#pragma unroll
+    for (int u = 0; u < kLd; ++u) {
+      const int t = t0 + u * kCsThreads;
+      if (t < nt) tile[t] = v[u];
+    }
   }
   __syncthreads();
-  for (int t = tid; t < n; t += kCsThreads) {
-    float pm = tile[t];
-    for (int o = 1; o <= 2 * r; ++o) pm = fmaxf(pm, tile[t + o]);
-    const float sc = __fsub_rn(__fmul_rn(lam, pm), __fmul_rn(one_minus_lam, rh[lo + t]));
-    if (score) score[(size_t)h * Lk + lo + t] = sc;
-    skeys[t] = order_key(sc);
+  for (int t0 = tid; t0 < n; t0 += kCsThreads * kLd) {
+    float rv[kLd];
+#pragma unroll
+    for (int u = 0; u < kLd; ++u) {
+      const int t = t0 + u * kCsThreads;
+      rv[u] = t < n ? rh[lo + t] : 0.0f;
+    }
+#pragma unroll
+    for (int u = 0; u < kLd; ++u) {
+      const int t = t0 + u * kCsThreads;
+      if (t < n) {
+        float pm = tile[t];
+        for (int o = 1; o <= 2 * r; ++o) pm = fmaxf(pm, tile[t + o]);
+        const float sc = __fsub_rn(__fmul_rn(lam, pm), __fmul_rn(one_minus_lam, rv[u]));
+        if (score) score[(size_t)h * Lk + lo + t] = sc;
+        skeys[t] = order_key(sc);
+      }
+    }
   }
   if (tid == 0) {
     s_prefix = 0u;
@@ -287,8 +313,14 @@ __global__ void __launch_bounds__(kCsThreads)
     }
     cluster.sync();
     if (tid < 256) {
+      // every CTA's count of this bin, all loads in flight before the sum
+      unsigned c[kCsMaxCluster];
+#pragma unroll
+      for (int q = 0; q < kCsMaxCluster; ++q)
+        c[q] = q < nrank ? *cluster.map_shared_rank(&hist[pass & 1][tid], q) : 0u;
       unsigned t = 0u;
-      for (int q = 0; q < nrank; ++q) t += *cluster.map_shared_rank(&hist[pass & 1][tid], q);
+#pragma unroll
+      for (int q = 0; q < kCsMaxCluster; ++q) t += c[q];
       s_total[tid] = t;
     }
     __syncthreads();
@@ -353,11 +385,21 @@ __global__ void __launch_bounds__(kCsThreads)
     s_cnt[1] = b;
   }
   cluster.sync();
-  // Counts of the CTAs before this one (their tokens come first).
+  // Counts of the CTAs before this one (their tokens come first), all loads
+  // in flight before the sums.
   int gt_base = 0, tie_base = 0;
-  for (int q = 0; q < rank; ++q) {
-    gt_base += *cluster.map_shared_rank(&s_cnt[0], q);
-    tie_base += *cluster.map_shared_rank(&s_cnt[1], q);
+  {
+    int cg_[kCsMaxCluster], ct_[kCsMaxCluster];
+#pragma unroll
+    for (int q = 0; q < kCsMaxCluster; ++q) {
+      cg_[q] = q < rank ? *cluster.map_shared_rank(&s_cnt[0], q) : 0;
+      ct_[q] = q < rank ? *cluster.map_shared_rank(&s_cnt[1], q) : 0;
+    }
+#pragma unroll
+    for (int q = 0; q < kCsMaxCluster; ++q) {
+      gt_base += cg_[q];
+      tie_base += ct_[q];
+    }
   }
   for (int w = 0; w < warp; ++w) {
     gt_base += s_wgt[w];

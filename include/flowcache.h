@@ -280,11 +280,17 @@ size_t fc_redundancy_workspace_size(fc_dtype dtype, int H, int Lk, int d);
  * column means of the cosine-similarity matrix with its diagonal zeroed.
  * Evaluated with the exact identity sum_{i != j} khat_i.khat_j =
  * khat_j.(sum_i khat_i) - ||khat_j||^2, so that K is streamed instead of the
- * Lk x Lk matrix being formed.
+ * Lk x Lk matrix being formed.  The sums over a head's keys (of khat, and of
+ * exp(r_j) for the softmax) are accumulated in 2^-32 fixed point in 64-bit
+ * integers, so the result is bitwise the same whatever the order in which
+ * the GPU finishes the pieces, and does not depend on H.  Heads are processed
+ * in groups whose keys fit in L2, so that the second read of K comes from L2.
  *
  *   k    [H][Lk][d] dtype
  *   red  [H][Lk] float32, out; each row sums to 1
- * Errors as for fc_kv_importance.
+ *   ws   fc_redundancy_workspace_size() bytes; no contents carried between
+ *        calls (the call clears what it uses)
+ * Errors as for fc_kv_importance; Lk > 2^26 -> FC_ERR_UNSUPPORTED.
  */
 fc_status fc_kv_redundancy(const void* k, fc_dtype dtype, int H, int Lk, int d, float* red,
                            void* ws, size_t ws_bytes, void* stream);
