@@ -14,8 +14,9 @@
 // thread keeps eight loads in flight, and the first of them go out before the
 // chunk's step counter and dt are read.  (Staging the stream through shared
 // memory with 1-D TMA bulk copies, one CTA per SM, measured 14% slower at 4
-// chunks and 6% slower at 16 on B200.)  Partial sums are float64 (exact enough that the float32 L1_rel is
-// practically the correctly rounded quotient).  Each block stores its partial
+// chunks and 6% slower at 16 on B200.)  The four magnitudes of a vector are
+// added in float32, the rest in float64, so the float32 L1_rel is within
+// 2^-23 relative of the exact quotient.  Each block stores its partial
 // pair; the last block of a chunk to finish (an integer completion counter,
 // no spinning, no float atomics) sums the partials in a fixed order and runs
 // the recurrence, so the result is deterministic and one launch does it all.

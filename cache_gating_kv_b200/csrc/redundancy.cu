@@ -80,16 +80,42 @@ __device__ __forceinline__ float row_sum(float v) {
   return v;
 }
 
+#ifndef FC_RED_L2HINT
+#define FC_RED_L2HINT 0
+#endif
+// 16-byte read-only load that does not allocate in L1, with an L2 cache policy
+// (evict_last for the first read of a key, evict_first for its last read).
+__device__ __forceinline__ uint4 ld_nc_v4_pol(const void* p, uint64_t pol) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0,%1,%2,%3}, [%4], %5;"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p), "l"(pol));
+  return r;
+}
+__device__ __forceinline__ uint64_t l2_policy(bool keep) {
+  uint64_t pol;
+  if (keep)
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  else
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 template <typename T, int D, int U>
 __device__ __forceinline__ void load_rows(const T* kh, int r0, int hi, int sub, int cl,
-                                          uint4 (&u)[U][2]) {
+                                          uint4 (&u)[U][2], uint64_t pol) {
   using L = RowLayout<T, D>;
 #pragma unroll
   for (int i = 0; i < U; ++i) {
     const int r = r0 + i * L::RPW + sub;
     const T* p = kh + (size_t)r * D + cl * L::EPL;
-    u[i][0] = r < hi ? ld_nc_v4(p) : make_uint4(0u, 0u, 0u, 0u);
-    u[i][1] = r < hi ? ld_nc_v4(p + Vec16<T>::N) : make_uint4(0u, 0u, 0u, 0u);
+    if (FC_RED_L2HINT) {
+      u[i][0] = r < hi ? ld_nc_v4_pol(p, pol) : make_uint4(0u, 0u, 0u, 0u);
+      u[i][1] = r < hi ? ld_nc_v4_pol(p + Vec16<T>::N, pol) : make_uint4(0u, 0u, 0u, 0u);
+    } else {
+      u[i][0] = r < hi ? ld_nc_v4(p) : make_uint4(0u, 0u, 0u, 0u);
+      u[i][1] = r < hi ? ld_nc_v4(p + Vec16<T>::N) : make_uint4(0u, 0u, 0u, 0u);
+    }
   }
 }
 
@@ -154,12 +180,13 @@ __global__ void __launch_bounds__(kRedThreads)
   __shared__ double s_esum[kRedWarps];
 
   if (phase == 1) {  // ---- sum of the slice's normalised rows ----------------
+    const uint64_t pol = FC_RED_L2HINT ? l2_policy(true) : 0ull;
     float a[L::EPL];
 #pragma unroll
     for (int i = 0; i < L::EPL; ++i) a[i] = 0.0f;
     for (int r0 = lo + warp * L::RPW * U; r0 < hi; r0 += kRowsPerIter) {
       uint4 raw[U][2];
-      load_rows<T, D, U>(kh, r0, hi, sub, cl, raw);
+      load_rows<T, D, U>(kh, r0, hi, sub, cl, raw, pol);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         float e[L::EPL];
@@ -199,10 +226,11 @@ __global__ void __launch_bounds__(kRedThreads)
 #pragma unroll
     for (int i = 0; i < L::EPL; ++i) sv[i] = s_vec[cl * L::EPL + i];
     const float inv_lk = 1.0f / (float)Lk;
+    const uint64_t pol = FC_RED_L2HINT ? l2_policy(false) : 0ull;
     double esum = 0.0;
     for (int r0 = lo + warp * L::RPW * U; r0 < hi; r0 += kRowsPerIter) {
       uint4 raw[U][2];
-      load_rows<T, D, U>(kh, r0, hi, sub, cl, raw);
+      load_rows<T, D, U>(kh, r0, hi, sub, cl, raw, pol);
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         float e[L::EPL];

@@ -235,6 +235,11 @@ __global__ void __launch_bounds__(kCsThreads)
   __shared__ int s_remaining;
   __shared__ int s_cnt[2];   // this CTA's (greater, tie) counts (read by the cluster)
   __shared__ int s_wgt[kCsWarps], s_wtie[kCsWarps];
+  __shared__ int s_ncand;
+
+  // The first radix pass's histogram (top 8 bits) is built while the keys
+  // are formed.
+  for (int i = tid; i < kCsWarps * 256; i += kCsThreads) (&whist[0][0])[i] = 0u;
 
   // ---- scores of the slice -> order-preserving keys ------------------------
   // Imp and Red were just written by the kernels before: each thread issues
@@ -257,7 +262,9 @@ __global__ void __launch_bounds__(kCsThreads)
     }
   }
   __syncthreads();
-  for (int t0 = tid; t0 < n; t0 += kCsThreads * kLd) {
+  // warp-uniform loop bounds: every lane takes part in the histogram's votes
+  for (int b0 = warp * 32; b0 < n; b0 += kCsThreads * kLd) {
+    const int t0 = b0 + lane;
     float rv[kLd];
 #pragma unroll
     for (int u = 0; u < kLd; ++u) {
@@ -267,12 +274,20 @@ __global__ void __launch_bounds__(kCsThreads)
 #pragma unroll
     for (int u = 0; u < kLd; ++u) {
       const int t = t0 + u * kCsThreads;
+      uint32_t key = 0u;
       if (t < n) {
         float pm = tile[t];
         for (int o = 1; o <= 2 * r; ++o) pm = fmaxf(pm, tile[t + o]);
         const float sc = __fsub_rn(__fmul_rn(lam, pm), __fmul_rn(one_minus_lam, rv[u]));
         if (score) score[(size_t)h * Lk + lo + t] = sc;
-        skeys[t] = order_key(sc);
+        key = order_key(sc);
+        skeys[t] = key;
+      }
+      const unsigned vm = __ballot_sync(0xffffffffu, t < n);
+      if (t < n) {
+        const unsigned digit = key >> 24;
+        const unsigned peers = __match_any_sync(vm, digit);
+        if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&whist[warp][digit], __popc(peers));
       }
     }
   }
@@ -284,27 +299,54 @@ __global__ void __launch_bounds__(kCsThreads)
   __syncthreads();
 
   // ---- 4 radix passes over the cluster's keys ----------------------------------
+  // Pass 0's histogram is already built.  Once two passes have fixed the top
+  // 16 bits of the threshold, the keys that still match them (a small part of
+  // the slice) are gathered into `cand` (the pooling tile's space, free by
+  // then) and the last two passes count only those.
+  uint32_t* cand = reinterpret_cast<uint32_t*>(tile);
+  const uint32_t* src = skeys;
+  int nsrc = n;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
     const uint32_t prefix = s_prefix, pmask = s_pmask;
-    for (int i = tid; i < kCsWarps * 256; i += kCsThreads) (&whist[0][0])[i] = 0u;
-    __syncthreads();
-    for (int j0 = warp * 32; j0 < n; j0 += kCsThreads) {
-      const int j = j0 + lane;
-      uint32_t key = 0u;
-      bool in = false;
-      if (j < n) {
-        key = skeys[j];
-        in = (key & pmask) == prefix;
+    if (pass == 2) {
+      if (tid == 0) s_ncand = 0;
+      __syncthreads();
+      const unsigned lt = (1u << lane) - 1u;
+      for (int j0 = warp * 32; j0 < n; j0 += kCsThreads) {
+        const int j = j0 + lane;
+        const uint32_t key = j < n ? skeys[j] : 0u;
+        const bool in = j < n && (key & pmask) == prefix;
+        const unsigned b = __ballot_sync(0xffffffffu, in);
+        int off = 0;
+        if (lane == 0 && b) off = atomicAdd(&s_ncand, __popc(b));
+        off = __shfl_sync(0xffffffffu, off, 0);
+        if (in) cand[off + __popc(b & lt)] = key;
       }
-      const unsigned vm = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const unsigned digit = (key >> shift) & 0xffu;
-        const unsigned peers = __match_any_sync(vm, digit);
-        if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&whist[warp][digit], __popc(peers));
-      }
+      __syncthreads();
+      src = cand;
+      nsrc = s_ncand;
     }
-    __syncthreads();
+    if (pass > 0) {
+      for (int i = tid; i < kCsWarps * 256; i += kCsThreads) (&whist[0][0])[i] = 0u;
+      __syncthreads();
+      for (int j0 = warp * 32; j0 < nsrc; j0 += kCsThreads) {
+        const int j = j0 + lane;
+        uint32_t key = 0u;
+        bool in = false;
+        if (j < nsrc) {
+          key = src[j];
+          in = (key & pmask) == prefix;
+        }
+        const unsigned vm = __ballot_sync(0xffffffffu, in);
+        if (in) {
+          const unsigned digit = (key >> shift) & 0xffu;
+          const unsigned peers = __match_any_sync(vm, digit);
+          if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&whist[warp][digit], __popc(peers));
+        }
+      }
+      __syncthreads();
+    }
     if (tid < 256) {  // one thread per bin
       unsigned t = 0u;
 #pragma unroll

@@ -65,3 +65,28 @@ def test_noalloc_gate_word_reads_the_static_scratch():
     mask = torch.empty(n_c, dtype=torch.uint8, device=DEV)
     fc.fc_chunk_l1_gate_noalloc(x, v, dt, st, 2, 0.05, f, l1, mask)
     assert fc.fc_check_workspace(fc.FC_WS_GATE_NOALLOC, None, n_c)
+
+
+def test_gates_reject_overlapping_latents_before_launching():
+    """x is updated in place while v is read (h_old overwritten while h_new is
+    read): any overlap of the two [n][N] arrays is refused on the host, and
+    nothing is written."""
+    n_c, N = 3, 4096
+    buf = torch.randn(n_c * N + 4, device=DEV)
+    x = buf[:n_c * N].view(n_c, N)
+    v_overlap = buf[4:].view(n_c, N)  # 16 bytes in: aligned, partly aliased
+    before = buf.clone()
+    dt = torch.full((n_c,), -0.1, device=DEV)
+    st = torch.full((n_c,), 3, dtype=torch.int32, device=DEV)
+    f = torch.zeros(n_c, device=DEV)
+    l1 = torch.full((n_c,), -1.0, device=DEV)
+    mask = torch.full((n_c,), 7, dtype=torch.uint8, device=DEV)
+    ws = fc.workspace(fc.fc_gate_workspace_size(n_c, N))
+    for call in (lambda: fc.fc_chunk_l1_gate(x, v_overlap, dt, st, 2, 0.05, f, l1, mask, ws),
+                 lambda: fc.fc_chunk_l1_gate_noalloc(x, v_overlap, dt, st, 2, 0.05, f, l1, mask),
+                 lambda: fc.fc_history_l1_gate(x, v_overlap, st, 2, 0.05, f, l1, mask, ws)):
+        with pytest.raises(fc.FlowCacheError) as e:
+            call()
+        assert e.value.status == 1 and "overlap" in str(e.value)
+    torch.cuda.synchronize()
+    assert torch.equal(buf, before) and float(l1[0]) == -1.0 and int(mask[0]) == 7
