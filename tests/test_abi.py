@@ -91,6 +91,9 @@ def test_kv_calls_reject_bad_shapes():
     assert lib.fc_kv_importance(NULL, NULL, fc.FC_BF16, 2, 0, 8, 64, 0.0, NULL, NULL, 0, NULL) == 1
     # unknown dtype
     assert lib.fc_kv_redundancy(NULL, 7, 2, 8, 64, NULL, NULL, 0, NULL) == 1
+    # more keys than the redundancy's fixed-point sums serve (2^26)
+    assert lib.fc_kv_redundancy(NULL, fc.FC_BF16, 1, (1 << 26) + 1, 64, NULL, NULL, 0, NULL) == 2
+    assert b"2^26" in lib.fc_last_error() or b"67108864" in lib.fc_last_error()
     # workspace too small
     assert lib.fc_kv_importance(NULL, NULL, fc.FC_BF16, 2, 8, 8, 64, 0.0, NULL, NULL, 4, NULL) == 3
     # score/top-B: B < 1, even or too wide pool window
