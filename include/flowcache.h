@@ -284,7 +284,7 @@ size_t fc_redundancy_workspace_size(fc_dtype dtype, int H, int Lk, int d);
  * exp(r_j) for the softmax) are accumulated in 2^-32 fixed point in 64-bit
  * integers, so the result is bitwise the same whatever the order in which
  * the GPU finishes the pieces, and does not depend on H.  Heads are processed
- * in groups whose keys fit in L2, so that the second read of K comes from L2.
+ * in groups, one group's sum overlapping the previous group's logits.
  *
  *   k    [H][Lk][d] dtype
  *   red  [H][Lk] float32, out; each row sums to 1
