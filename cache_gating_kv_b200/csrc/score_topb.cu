@@ -203,17 +203,37 @@ __global__ void __launch_bounds__(kSelThreads)
 // histograms through distributed shared memory (every CTA derives the same
 // digit), and the final ordered compaction offsets each CTA by the kept
 // counts of the CTAs before it.  Cluster barriers are hardware barriers.
+//
+// Two shapes.  8-CTA clusters (L_k <= 32768): 512-thread CTAs, a histogram
+// per warp, the whole slice's pooling tile at once.  16-CTA clusters: 256
+// threads, four shared histograms, the pooling tile in sub-tiles of 1024
+// keys, so that a CTA needs about 44 KB of shared memory and 40 heads' 640
+// CTAs are all resident at once (with 512 threads and the whole tile, 85 KB
+// per CTA, they ran in three waves: 31 us per CTA, ~110 us per call).
 // ---------------------------------------------------------------------------
-constexpr int kCsThreads = 512;  // 256 measured 8 % (L_k 16384) to 27 % (131072) slower
-constexpr int kCsWarps = kCsThreads / 32;
-static_assert(kCsThreads >= 256, "one thread per histogram bin");
 constexpr int kCsMaxSlice = 12288;  // keys per CTA held in shared memory
 constexpr int kCsMaxCluster = 16;   // CTAs per cluster (one head)
+constexpr int kCsSubKeys = 1024;    // keys per pooling sub-tile (16-CTA shape)
 
-__global__ void __launch_bounds__(kCsThreads)
+// kThreads: CTA size; kHists: histogram copies (one per warp, or fewer shared
+// by several warps); kSub: the pooling tile covers kCsSubKeys keys at a time
+// instead of the whole slice.
+// Resident CTAs per SM each shape is compiled for (registers capped to fit):
+// three 512-thread CTAs keep 40 heads' 320 CTAs of the 8-CTA shape in one
+// wave (at 59 registers two fit, and the call took 46 instead of 34 us).
+template <int kThreads>
+constexpr int cs_min_blocks() {
+  return kThreads == 512 ? 3 : 5;
+}
+
+template <int kThreads, int kHists, bool kSub>
+__global__ void __launch_bounds__(kThreads, cs_min_blocks<kThreads>())
     score_select_cluster_kernel(const float* __restrict__ imp, const float* __restrict__ red,
                                 int Lk, int r, float lam, float one_minus_lam, int B,
                                 float* __restrict__ score, int32_t* __restrict__ idx) {
+  static_assert(kThreads >= 256, "one thread per histogram bin");
+  constexpr int kWarps = kThreads / 32;
+  static_assert(kWarps % kHists == 0, "warps share histograms evenly");
   grid_dep_wait();  // the kernel before this one (importance) has finished
   grid_dep_launch();
   cg::cluster_group cluster = cg::this_cluster();
@@ -224,22 +244,24 @@ __global__ void __launch_bounds__(kCsThreads)
   const int per = (int)ceil_div(Lk, nrank);
   const int lo = min(Lk, rank * per), hi = min(Lk, lo + per);
   const int n = hi - lo;
+  const int tkeys = kSub ? kCsSubKeys : per;  // keys the pooling tile covers at once
 
   extern __shared__ __align__(16) unsigned char csm[];
   uint32_t* skeys = reinterpret_cast<uint32_t*>(csm);          // [per]
-  float* tile = reinterpret_cast<float*>(csm + (size_t)per * 4);  // [per + 2r]
-  __shared__ unsigned whist[kCsWarps][256];
+  float* tile = reinterpret_cast<float*>(csm + (size_t)per * 4);  // [tkeys + 2r]
+  __shared__ unsigned whist[kHists][256];
   __shared__ unsigned hist[2][256];  // this CTA's histogram, double-buffered by pass
   __shared__ unsigned s_total[256];
   __shared__ uint32_t s_prefix, s_pmask;
   __shared__ int s_remaining;
   __shared__ int s_cnt[2];   // this CTA's (greater, tie) counts (read by the cluster)
-  __shared__ int s_wgt[kCsWarps], s_wtie[kCsWarps];
+  __shared__ int s_wgt[kWarps], s_wtie[kWarps];
   __shared__ int s_ncand;
+  unsigned* myhist = whist[warp % kHists];
 
   // The first radix pass's histogram (top 8 bits) is built while the keys
   // are formed.
-  for (int i = tid; i < kCsWarps * 256; i += kCsThreads) (&whist[0][0])[i] = 0u;
+  for (int i = tid; i < kHists * 256; i += kThreads) (&whist[0][0])[i] = 0u;
 
   // ---- scores of the slice -> order-preserving keys ------------------------
   // Imp and Red were just written by the kernels before: each thread issues
@@ -247,47 +269,51 @@ __global__ void __launch_bounds__(kCsThreads)
   constexpr int kLd = 8;
   const float* ih = imp + (size_t)h * Lk;
   const float* rh = red + (size_t)h * Lk;
-  const int nt = n + 2 * r;
-  for (int t0 = tid; t0 < nt; t0 += kCsThreads * kLd) {
-    float v[kLd];
+  for (int base = 0; base < n; base += tkeys) {
+    const int m = min(tkeys, n - base);  // keys of this tile
+    const int nt = m + 2 * r;
+    if (base > 0) __syncthreads();  // the previous tile has been used
+    for (int t0 = tid; t0 < nt; t0 += kThreads * kLd) {
+      float v[kLd];
 #pragma unroll
-    for (int u = 0; u < kLd; ++u) {
-      const int t = t0 + u * kCsThreads, j = lo - r + t;
-      v[u] = (t < nt && j >= 0 && j < Lk) ? ih[j] : -INFINITY;  // out-of-range taps ignored
-    }
-#pragma unroll
-    for (int u = 0; u < kLd; ++u) {
-      const int t = t0 + u * kCsThreads;
-      if (t < nt) tile[t] = v[u];
-    }
-  }
-  __syncthreads();
-  // warp-uniform loop bounds: every lane takes part in the histogram's votes
-  for (int b0 = warp * 32; b0 < n; b0 += kCsThreads * kLd) {
-    const int t0 = b0 + lane;
-    float rv[kLd];
-#pragma unroll
-    for (int u = 0; u < kLd; ++u) {
-      const int t = t0 + u * kCsThreads;
-      rv[u] = t < n ? rh[lo + t] : 0.0f;
-    }
-#pragma unroll
-    for (int u = 0; u < kLd; ++u) {
-      const int t = t0 + u * kCsThreads;
-      uint32_t key = 0u;
-      if (t < n) {
-        float pm = tile[t];
-        for (int o = 1; o <= 2 * r; ++o) pm = fmaxf(pm, tile[t + o]);
-        const float sc = __fsub_rn(__fmul_rn(lam, pm), __fmul_rn(one_minus_lam, rv[u]));
-        if (score) score[(size_t)h * Lk + lo + t] = sc;
-        key = order_key(sc);
-        skeys[t] = key;
+      for (int u = 0; u < kLd; ++u) {
+        const int t = t0 + u * kThreads, j = lo + base - r + t;
+        v[u] = (t < nt && j >= 0 && j < Lk) ? ih[j] : -INFINITY;  // out-of-range taps ignored
       }
-      const unsigned vm = __ballot_sync(0xffffffffu, t < n);
-      if (t < n) {
-        const unsigned digit = key >> 24;
-        const unsigned peers = __match_any_sync(vm, digit);
-        if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&whist[warp][digit], __popc(peers));
+#pragma unroll
+      for (int u = 0; u < kLd; ++u) {
+        const int t = t0 + u * kThreads;
+        if (t < nt) tile[t] = v[u];
+      }
+    }
+    __syncthreads();
+    // warp-uniform loop bounds: every lane takes part in the histogram's votes
+    for (int b0 = warp * 32; b0 < m; b0 += kThreads * kLd) {
+      const int t0 = b0 + lane;
+      float rv[kLd];
+#pragma unroll
+      for (int u = 0; u < kLd; ++u) {
+        const int t = t0 + u * kThreads;
+        rv[u] = t < m ? rh[lo + base + t] : 0.0f;
+      }
+#pragma unroll
+      for (int u = 0; u < kLd; ++u) {
+        const int t = t0 + u * kThreads;
+        uint32_t key = 0u;
+        if (t < m) {
+          float pm = tile[t];
+          for (int o = 1; o <= 2 * r; ++o) pm = fmaxf(pm, tile[t + o]);
+          const float sc = __fsub_rn(__fmul_rn(lam, pm), __fmul_rn(one_minus_lam, rv[u]));
+          if (score) score[(size_t)h * Lk + lo + base + t] = sc;
+          key = order_key(sc);
+          skeys[base + t] = key;
+        }
+        const unsigned vm = __ballot_sync(0xffffffffu, t < m);
+        if (t < m) {
+          const unsigned digit = key >> 24;
+          const unsigned peers = __match_any_sync(vm, digit);
+          if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&myhist[digit], __popc(peers));
+        }
       }
     }
   }
@@ -302,8 +328,10 @@ __global__ void __launch_bounds__(kCsThreads)
   // Pass 0's histogram is already built.  Once two passes have fixed the top
   // 16 bits of the threshold, the keys that still match them (a small part of
   // the slice) are gathered into `cand` (the pooling tile's space, free by
-  // then) and the last two passes count only those.
+  // then) and the last two passes count only those; if more match than the
+  // space holds, the last passes scan the whole slice instead.
   uint32_t* cand = reinterpret_cast<uint32_t*>(tile);
+  const int cand_cap = tkeys + 2 * r;
   const uint32_t* src = skeys;
   int nsrc = n;
   for (int pass = 0; pass < 4; ++pass) {
@@ -313,7 +341,7 @@ __global__ void __launch_bounds__(kCsThreads)
       if (tid == 0) s_ncand = 0;
       __syncthreads();
       const unsigned lt = (1u << lane) - 1u;
-      for (int j0 = warp * 32; j0 < n; j0 += kCsThreads) {
+      for (int j0 = warp * 32; j0 < n; j0 += kThreads) {
         const int j = j0 + lane;
         const uint32_t key = j < n ? skeys[j] : 0u;
         const bool in = j < n && (key & pmask) == prefix;
@@ -321,16 +349,19 @@ __global__ void __launch_bounds__(kCsThreads)
         int off = 0;
         if (lane == 0 && b) off = atomicAdd(&s_ncand, __popc(b));
         off = __shfl_sync(0xffffffffu, off, 0);
-        if (in) cand[off + __popc(b & lt)] = key;
+        const int pos = off + __popc(b & lt);
+        if (in && pos < cand_cap) cand[pos] = key;
       }
       __syncthreads();
-      src = cand;
-      nsrc = s_ncand;
+      if (s_ncand <= cand_cap) {
+        src = cand;
+        nsrc = s_ncand;
+      }
     }
     if (pass > 0) {
-      for (int i = tid; i < kCsWarps * 256; i += kCsThreads) (&whist[0][0])[i] = 0u;
+      for (int i = tid; i < kHists * 256; i += kThreads) (&whist[0][0])[i] = 0u;
       __syncthreads();
-      for (int j0 = warp * 32; j0 < nsrc; j0 += kCsThreads) {
+      for (int j0 = warp * 32; j0 < nsrc; j0 += kThreads) {
         const int j = j0 + lane;
         uint32_t key = 0u;
         bool in = false;
@@ -342,7 +373,7 @@ __global__ void __launch_bounds__(kCsThreads)
         if (in) {
           const unsigned digit = (key >> shift) & 0xffu;
           const unsigned peers = __match_any_sync(vm, digit);
-          if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&whist[warp][digit], __popc(peers));
+          if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&myhist[digit], __popc(peers));
         }
       }
       __syncthreads();
@@ -350,7 +381,7 @@ __global__ void __launch_bounds__(kCsThreads)
     if (tid < 256) {  // one thread per bin
       unsigned t = 0u;
 #pragma unroll
-      for (int w = 0; w < kCsWarps; ++w) t += whist[w][tid];
+      for (int w = 0; w < kHists; ++w) t += whist[w][tid];
       hist[pass & 1][tid] = t;
     }
     cluster.sync();
@@ -403,7 +434,7 @@ __global__ void __launch_bounds__(kCsThreads)
   // ---- ordered compaction: keep every key > T and the first `need` keys == T ----
   const uint32_t T = s_prefix;
   const int need = s_remaining;
-  const int seg = (int)ceil_div(ceil_div(n, kCsWarps), 32) * 32;
+  const int seg = (int)ceil_div(ceil_div(n, kWarps), 32) * 32;
   const int w_lo = min(n, warp * seg), w_hi = min(n, w_lo + seg);
   int gt = 0, tie = 0;
   for (int j0 = w_lo; j0 < w_hi; j0 += 32) {
@@ -419,7 +450,7 @@ __global__ void __launch_bounds__(kCsThreads)
   __syncthreads();
   if (tid == 0) {
     int a = 0, b = 0;
-    for (int w = 0; w < kCsWarps; ++w) {
+    for (int w = 0; w < kWarps; ++w) {
       a += s_wgt[w];
       b += s_wtie[w];
     }
@@ -486,21 +517,30 @@ cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk,
   const float one_minus = 1.0f - lambda;  // float32, as the score's definition
   const int r = pool / 2;
   if (B < Lk && Lk <= 16 * kCsMaxSlice) {
-    // One cluster per head: 8 CTAs, or 16 (non-portable) for long histories.
-    const int csize = Lk > 8 * 4096 ? 16 : 8;
+    // One cluster per head: 8 CTAs of 512 threads, or 16 (non-portable) of
+    // 256 threads with sub-tiled pooling for long histories.
+    const bool large = Lk > 8 * 4096;
+    const int csize = large ? 16 : 8;
+    const int threads = large ? 256 : 512;
     const int per = (int)ceil_div(Lk, csize);
-    const size_t smem = (size_t)per * 4 + (size_t)(per + 2 * r) * 4;
-    auto kern = score_select_cluster_kernel;
+    const int tkeys = large ? kCsSubKeys : per;
+    const size_t smem = (size_t)per * 4 + (size_t)(tkeys + 2 * r) * 4;
+    auto kern = large ? score_select_cluster_kernel<256, 4, true>
+                      : score_select_cluster_kernel<512, 16, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     if (csize > 8) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e != cudaSuccess) return e;
+      // all of the SM's shared memory, so that five ~45 KB CTAs fit on an SM
+      e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                               cudaSharedmemCarveoutMaxShared);
+      if (e != cudaSuccess) return e;
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)csize, (unsigned)H, 1);
-    cfg.blockDim = dim3(kCsThreads, 1, 1);
+    cfg.blockDim = dim3((unsigned)threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];
