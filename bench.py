@@ -230,22 +230,23 @@ def bench_config(workload, per_rank="one independent layer per GPU"):
             "l2": "flushed between steps (256 MiB write + read-back, outside the timed events)"}
 
 
-# DRAM bytes (read + write) of one fc_kv_importance call, per head, from one
-# ncu capture of its launches (dram__bytes_read.sum + dram__bytes_write.sum) on
-# a subset of the workload's heads: workload -> (bytes per head, heads captured).
-# The traffic of the call grows in proportion to its heads (every head is an
-# independent slab of Q and K), so a full call is heads x the per-head bytes.
-# Keep in step with the kernel: a change to the importance kernels voids it.
-IMP_TRAFFIC_PER_HEAD = {
+# DRAM bytes (read + write) of one fc_kv_importance call over a workload's
+# heads, from one ncu capture of its launches (dram__bytes_read.sum +
+# dram__bytes_write.sum): workload -> (bytes per call, heads in the call).  The
+# bytes per head depend on how many heads' keys are in flight at once (4 heads
+# read Q and K exactly once per pass, 12 and 40 heads 1.17-1.24x in the row
+# pass), so the figure holds only for the head count it was taken at; any
+# other count reports null.  A change to the importance kernels voids it.
+IMP_TRAFFIC = {
     # all 40 heads captured at once (the three metrics take one ncu pass):
     # row pass 1662.2 + 12.9 MB, column pass 1438.9 + 20.4 MB
-    "long_history": (3134.4e6 / 40, 40),
+    "long_history": (3134.4e6, 40),
 }
 
 
 def _traffic(workload, H):
-    t = IMP_TRAFFIC_PER_HEAD.get(workload)
-    return None if t is None else t[0] * H
+    t = IMP_TRAFFIC.get(workload)
+    return t[0] if t is not None and t[1] == H else None
 
 
 class Step:
@@ -530,7 +531,7 @@ def native(a, rank, world, local_rank):
                      "frac_of_sustained_peak": imp_tf / tf_sus,
                      "traffic": _traffic(a.workload, H),
                      "traffic_unit": "bytes per call (DRAM read + write of the call's "
-                                     "launches, from one ncu capture, scaled by heads)"},
+                                     "launches, from one ncu capture of this workload)"},
         "kernels_ms": ms_call,
         "kernels_ms_alone": ms_alone,
         "kernels_note": "kernels_ms: spans inside the timed step (gate and redundancy share "
@@ -665,11 +666,10 @@ def _full_step_sweep(dev, stream, side, flush, sink, seed, lk=131072, layers=40,
     apiece, ten times the L2, so no layer finds the previous one's data in
     cache (at L_k = 4096 a layer's K is 42 MB, and the alternation keeps the
     two layers apart by one layer's traffic)."""
+    import cache_gating_kv_b200 as fc
     from cache_gating_kv_b200 import workloads as W
 
     kv, gc = W.KV_CONFIGS[f"sweep_lk{lk}"], W.GATE_CONFIGS["full_step_sweep"]
-    import cache_gating_kv_b200 as fc
-
     ls = [Step(kv, None, seed=seed, dev=dev, layer=i) for i in range(2)]
     g = _gate_bufs(gc, seed, dev)
     ev0 = torch.cuda.Event(enable_timing=True)

@@ -352,7 +352,6 @@ fc_status fc_kv_importance(const void* q, const void* k, fc_dtype dtype, int H, 
 
 size_t fc_redundancy_workspace_size(fc_dtype dtype, int H, int Lk, int d) {
   (void)dtype;
-  (void)Lk;
   return (H < 1 || Lk < 1 || (d != 64 && d != 128)) ? 0 : fc::redundancy_ws_bytes(H, Lk, d);
 }
 
