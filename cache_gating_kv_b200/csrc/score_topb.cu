@@ -205,28 +205,33 @@ __global__ void __launch_bounds__(kSelThreads)
 // counts of the CTAs before it.  Cluster barriers are hardware barriers.
 //
 // Two shapes.  8-CTA clusters (L_k <= 32768): 512-thread CTAs, a histogram
-// per warp, the whole slice's pooling tile at once.  16-CTA clusters: 256
-// threads, four shared histograms, the pooling tile in sub-tiles of 1024
-// keys, so that a CTA needs about 44 KB of shared memory and 40 heads' 640
-// CTAs are all resident at once (with 512 threads and the whole tile, 85 KB
-// per CTA, they ran in three waves: 31 us per CTA, ~110 us per call).
+// per warp, the slice's pooling tile and its keys in separate buffers.
+// 16-CTA clusters: 256 threads, one histogram, and the keys written over the
+// pooling tile (each key over the tile position of its own first tap, a
+// chunk of 2048 keys at a time once the chunk's taps have been read), so that
+// a CTA needs about 37 KB of shared memory at L_k = 131072 and six fit on an
+// SM: 40 heads' 640 CTAs then run in one wave.  (With separate 1024-key
+// pooling sub-tiles, 44 KB and five per SM, the GPU held 38 such clusters at
+// once and the last two heads ran in a second wave: 124 us per call against
+// 49 us for four heads.)
 // ---------------------------------------------------------------------------
 constexpr int kCsMaxSlice = 12288;  // keys per CTA held in shared memory
 constexpr int kCsMaxCluster = 16;   // CTAs per cluster (one head)
-constexpr int kCsSubKeys = 1024;    // keys per pooling sub-tile (16-CTA shape)
+constexpr int kCsCandCap = 384;     // in-place shape: room for the last passes' candidates
 
 // kThreads: CTA size; kHists: histogram copies (one per warp, or fewer shared
-// by several warps); kSub: the pooling tile covers kCsSubKeys keys at a time
-// instead of the whole slice.
+// by several warps); kInPlace: the keys overwrite the pooling tile (and the
+// last passes' candidates get a small buffer of their own after it).
 // Resident CTAs per SM each shape is compiled for (registers capped to fit):
 // three 512-thread CTAs keep 40 heads' 320 CTAs of the 8-CTA shape in one
-// wave (at 59 registers two fit, and the call took 46 instead of 34 us).
+// wave (at 59 registers two fit, and the call took 46 instead of 34 us); six
+// 256-thread CTAs the 16-CTA shape's 640.
 template <int kThreads>
 constexpr int cs_min_blocks() {
-  return kThreads == 512 ? 3 : 5;
+  return kThreads == 512 ? 3 : 6;
 }
 
-template <int kThreads, int kHists, bool kSub>
+template <int kThreads, int kHists, bool kInPlace>
 __global__ void __launch_bounds__(kThreads, cs_min_blocks<kThreads>())
     score_select_cluster_kernel(const float* __restrict__ imp, const float* __restrict__ red,
                                 int Lk, int r, float lam, float one_minus_lam, int B,
@@ -244,14 +249,18 @@ __global__ void __launch_bounds__(kThreads, cs_min_blocks<kThreads>())
   const int per = (int)ceil_div(Lk, nrank);
   const int lo = min(Lk, rank * per), hi = min(Lk, lo + per);
   const int n = hi - lo;
-  const int tkeys = kSub ? kCsSubKeys : per;  // keys the pooling tile covers at once
 
+  // Separate buffers: keys [per], then the pooling tile [per + 2r].  In place:
+  // the pooling tile [per + 2r] whose first n positions end up holding the
+  // keys, then the candidate buffer [kCsCandCap].
   extern __shared__ __align__(16) unsigned char csm[];
-  uint32_t* skeys = reinterpret_cast<uint32_t*>(csm);          // [per]
-  float* tile = reinterpret_cast<float*>(csm + (size_t)per * 4);  // [tkeys + 2r]
+  uint32_t* skeys = reinterpret_cast<uint32_t*>(csm);
+  float* tile = reinterpret_cast<float*>(kInPlace ? csm : csm + (size_t)per * 4);
   __shared__ unsigned whist[kHists][256];
   __shared__ unsigned hist[2][256];  // this CTA's histogram, double-buffered by pass
-  __shared__ unsigned s_total[256];
+  // the cluster's totals of a pass: written after the pass's histograms have
+  // been folded into hist[] and read before they are cleared for the next
+  unsigned* s_total = &whist[0][0];
   __shared__ uint32_t s_prefix, s_pmask;
   __shared__ int s_remaining;
   __shared__ int s_cnt[2];   // this CTA's (greater, tie) counts (read by the cluster)
@@ -269,51 +278,62 @@ __global__ void __launch_bounds__(kThreads, cs_min_blocks<kThreads>())
   constexpr int kLd = 8;
   const float* ih = imp + (size_t)h * Lk;
   const float* rh = red + (size_t)h * Lk;
-  for (int base = 0; base < n; base += tkeys) {
-    const int m = min(tkeys, n - base);  // keys of this tile
-    const int nt = m + 2 * r;
-    if (base > 0) __syncthreads();  // the previous tile has been used
-    for (int t0 = tid; t0 < nt; t0 += kThreads * kLd) {
-      float v[kLd];
+  const int nt = n + 2 * r;
+  for (int t0 = tid; t0 < nt; t0 += kThreads * kLd) {
+    float v[kLd];
 #pragma unroll
-      for (int u = 0; u < kLd; ++u) {
-        const int t = t0 + u * kThreads, j = lo + base - r + t;
-        v[u] = (t < nt && j >= 0 && j < Lk) ? ih[j] : -INFINITY;  // out-of-range taps ignored
+    for (int u = 0; u < kLd; ++u) {
+      const int t = t0 + u * kThreads, j = lo - r + t;
+      v[u] = (t < nt && j >= 0 && j < Lk) ? ih[j] : -INFINITY;  // out-of-range taps ignored
+    }
+#pragma unroll
+    for (int u = 0; u < kLd; ++u) {
+      const int t = t0 + u * kThreads;
+      if (t < nt) tile[t] = v[u];
+    }
+  }
+  __syncthreads();
+  // Block-uniform loop over chunks of kThreads * kLd keys (every lane takes
+  // part in the histogram's votes, and the in-place shape's barrier is
+  // reached by every thread).  Key t reads taps t .. t + 2r of the tile.
+  for (int c0 = 0; c0 < n; c0 += kThreads * kLd) {
+    const int t0 = c0 + warp * 32 + lane;
+    float rv[kLd];
+#pragma unroll
+    for (int u = 0; u < kLd; ++u) {
+      const int t = t0 + u * kThreads;
+      rv[u] = t < n ? rh[lo + t] : 0.0f;
+    }
+    uint32_t kk[kLd];
+#pragma unroll
+    for (int u = 0; u < kLd; ++u) {
+      const int t = t0 + u * kThreads;
+      uint32_t key = 0u;
+      if (t < n) {
+        float pm = tile[t];
+        for (int o = 1; o <= 2 * r; ++o) pm = fmaxf(pm, tile[t + o]);
+        const float sc = __fsub_rn(__fmul_rn(lam, pm), __fmul_rn(one_minus_lam, rv[u]));
+        if (score) score[(size_t)h * Lk + lo + t] = sc;
+        key = order_key(sc);
+        if (!kInPlace) skeys[t] = key;
       }
-#pragma unroll
-      for (int u = 0; u < kLd; ++u) {
-        const int t = t0 + u * kThreads;
-        if (t < nt) tile[t] = v[u];
+      kk[u] = key;
+      const unsigned vm = __ballot_sync(0xffffffffu, t < n);
+      if (t < n) {
+        const unsigned digit = key >> 24;
+        const unsigned peers = __match_any_sync(vm, digit);
+        if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&myhist[digit], __popc(peers));
       }
     }
-    __syncthreads();
-    // warp-uniform loop bounds: every lane takes part in the histogram's votes
-    for (int b0 = warp * 32; b0 < m; b0 += kThreads * kLd) {
-      const int t0 = b0 + lane;
-      float rv[kLd];
+    if (kInPlace) {
+      // Every tap of this chunk has been read; its keys go over its first
+      // positions.  The next chunk reads taps from position c0 + kThreads*kLd
+      // on, which no key of this chunk overwrites.
+      __syncthreads();
 #pragma unroll
       for (int u = 0; u < kLd; ++u) {
         const int t = t0 + u * kThreads;
-        rv[u] = t < m ? rh[lo + base + t] : 0.0f;
-      }
-#pragma unroll
-      for (int u = 0; u < kLd; ++u) {
-        const int t = t0 + u * kThreads;
-        uint32_t key = 0u;
-        if (t < m) {
-          float pm = tile[t];
-          for (int o = 1; o <= 2 * r; ++o) pm = fmaxf(pm, tile[t + o]);
-          const float sc = __fsub_rn(__fmul_rn(lam, pm), __fmul_rn(one_minus_lam, rv[u]));
-          if (score) score[(size_t)h * Lk + lo + base + t] = sc;
-          key = order_key(sc);
-          skeys[base + t] = key;
-        }
-        const unsigned vm = __ballot_sync(0xffffffffu, t < m);
-        if (t < m) {
-          const unsigned digit = key >> 24;
-          const unsigned peers = __match_any_sync(vm, digit);
-          if ((unsigned)lane == (unsigned)(__ffs(peers) - 1)) atomicAdd(&myhist[digit], __popc(peers));
-        }
+        if (t < n) skeys[t] = kk[u];
       }
     }
   }
@@ -330,8 +350,8 @@ __global__ void __launch_bounds__(kThreads, cs_min_blocks<kThreads>())
   // the slice) are gathered into `cand` (the pooling tile's space, free by
   // then) and the last two passes count only those; if more match than the
   // space holds, the last passes scan the whole slice instead.
-  uint32_t* cand = reinterpret_cast<uint32_t*>(tile);
-  const int cand_cap = tkeys + 2 * r;
+  uint32_t* cand = kInPlace ? skeys + (per + 2 * r) : reinterpret_cast<uint32_t*>(tile);
+  const int cand_cap = kInPlace ? kCsCandCap : per + 2 * r;
   const uint32_t* src = skeys;
   int nsrc = n;
   for (int pass = 0; pass < 4; ++pass) {
@@ -523,9 +543,9 @@ cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk,
     const int csize = large ? 16 : 8;
     const int threads = large ? 256 : 512;
     const int per = (int)ceil_div(Lk, csize);
-    const int tkeys = large ? kCsSubKeys : per;
-    const size_t smem = (size_t)per * 4 + (size_t)(tkeys + 2 * r) * 4;
-    auto kern = large ? score_select_cluster_kernel<256, 4, true>
+    const size_t smem = large ? (size_t)(per + 2 * r + kCsCandCap) * 4
+                              : (size_t)per * 4 + (size_t)(per + 2 * r) * 4;
+    auto kern = large ? score_select_cluster_kernel<256, 1, true>
                       : score_select_cluster_kernel<512, 16, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -533,7 +553,7 @@ cudaError_t launch_score_topb(const float* imp, const float* red, int H, int Lk,
     if (csize > 8) {
       e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e != cudaSuccess) return e;
-      // all of the SM's shared memory, so that five ~45 KB CTAs fit on an SM
+      // all of the SM's shared memory, so that six ~37 KB CTAs fit on an SM
       e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
                                cudaSharedmemCarveoutMaxShared);
       if (e != cudaSuccess) return e;
