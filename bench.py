@@ -940,7 +940,7 @@ def main():
     try:
         out = native(a, rank, world, local_rank)
         if rank == 0:
-            if not a.no_cpu_baseline:
+            if not a.no_cpu_baseline and world == 1:  # the oracle's baseline: rank 0 at N=1
                 out["cpu_baseline"] = cpu_baseline(a)
             print(json.dumps(out))
     finally:
