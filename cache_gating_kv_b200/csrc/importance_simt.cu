@@ -7,16 +7,28 @@
 // queries.
 //
 // Two passes, both tiled 64 x 64 with a 4 x 4 register tile per thread:
-//   pass 1  grid (L_q/64, H): for a query tile, stream every key tile and keep
-//           a running (max, sum) per row in the log2 domain; store
-//           lse2_q = log2 sum_j 2^(c*s_qj) with c = scale*log2(e)
-//   pass 2  grid (L_k/64, H): for a key tile, stream every query tile and
-//           accumulate 2^(c*s_qj - lse2_q) per key; fixed-order reduction at
-//           the end, divided by L_q.  No atomics: each block owns its keys.
-// float32 accumulation throughout; exp2f / log2f are the accurate library
-// functions (this path carries the float32 tolerance).
+//   pass 1  one thread-block cluster of C1 CTAs per (query tile, head): CTA r
+//           streams the r-th share of the key tiles and keeps a running
+//           (max, sum) per row in the log2 domain; CTA 0 merges the C1 pairs
+//           of each row over distributed shared memory, in rank order, and
+//           stores lse2_q = log2 sum_j 2^(c*s_qj) with c = scale*log2(e)
+//   pass 2  one cluster of C2 CTAs per (key tile, head): CTA r streams the
+//           r-th share of the query tiles and accumulates 2^(c*s_qj - lse2_q)
+//           per key; CTA 0 adds the C2 partial sums in rank order and divides
+//           by L_q.  No atomics: each cluster owns its rows or keys.
+// C1 and C2 (at most 8) spread small problems over the SMs (the 2-head
+// parity case has 8 query tiles and 32 key tiles in all); they depend only on
+// the problem's size, so the result is the same on every run.  float32
+// accumulation throughout; exp2f / log2f are the accurate library functions
+// (this path carries the float32 tolerance).
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
 #include "fc_common.cuh"
 #include "fc_kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace fc {
 
@@ -67,6 +79,17 @@ __device__ __forceinline__ void tile_dot(const float* __restrict__ As, const flo
   }
 }
 
+// (max, sum) of two partial log2-domain sums merged; -inf max means empty.
+__device__ __forceinline__ void merge_ml(float& m, float& l, float mo, float lo) {
+  const float mn = fmaxf(m, mo);
+  if (mn != -INFINITY) {
+    const float a = (m == -INFINITY) ? 0.0f : l * exp2f(m - mn);
+    const float b = (mo == -INFINITY) ? 0.0f : lo * exp2f(mo - mn);
+    l = a + b;
+    m = mn;
+  }
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kThreads)
     imp_lse_simt(const T* __restrict__ q, const T* __restrict__ k, int Lq, int Lk, int ldk,
@@ -75,8 +98,13 @@ __global__ void __launch_bounds__(kThreads)
   extern __shared__ __align__(16) float sm[];
   float* Qs = sm;
   float* Ks = sm + D * kPad;
-  const int h = blockIdx.y, q0 = blockIdx.x * kT;
+  __shared__ float2 s_ml[kT];  // this CTA's (max, sum) per row of the query tile
+  cg::cluster_group cluster = cg::this_cluster();
+  const int nr = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
+  const int h = blockIdx.y, q0 = (blockIdx.x / nr) * kT;
   const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  const int nkt = (int)ceil_div(Lk, kT), per = (int)ceil_div(nkt, nr);
+  const int kt0 = rank * per, kt1 = min(nkt, kt0 + per);
   load_tile_t<T, D>(Qs, q + ((size_t)h * Lq + q0) * D, min(kT, Lq - q0));
   float m[4], l[4];
 #pragma unroll
@@ -84,7 +112,7 @@ __global__ void __launch_bounds__(kThreads)
     m[i] = -INFINITY;
     l[i] = 0.0f;
   }
-  for (int k0 = 0; k0 < Lk; k0 += kT) {
+  for (int k0 = kt0 * kT; k0 < kt1 * kT; k0 += kT) {
     __syncthreads();
     load_tile_t<T, D>(Ks, k + ((size_t)h * ldk + k0) * D, min(kT, Lk - k0));
     __syncthreads();
@@ -116,17 +144,22 @@ __global__ void __launch_bounds__(kThreads)
     for (int o = 8; o > 0; o >>= 1) {
       const float mo = __shfl_xor_sync(0xffffffffu, m[i], o);
       const float lo = __shfl_xor_sync(0xffffffffu, l[i], o);
-      const float mn = fmaxf(m[i], mo);
-      if (mn != -INFINITY) {
-        const float a = (m[i] == -INFINITY) ? 0.0f : l[i] * exp2f(m[i] - mn);
-        const float b = (mo == -INFINITY) ? 0.0f : lo * exp2f(mo - mn);
-        l[i] = a + b;
-        m[i] = mn;
-      }
+      merge_ml(m[i], l[i], mo, lo);
     }
-    const int row = q0 + ty * 4 + i;
-    if (tx == 0 && row < Lq) lse2[(size_t)h * Lq + row] = m[i] + log2f(l[i]);
+    if (tx == 0) s_ml[ty * 4 + i] = make_float2(m[i], l[i]);
   }
+  cluster.sync();
+  // CTA 0 merges the cluster's key shares of each row, in rank order.
+  if (rank == 0 && threadIdx.x < kT) {
+    float2 ml = s_ml[threadIdx.x];
+    for (int r = 1; r < nr; ++r) {
+      const float2 o = *cluster.map_shared_rank(&s_ml[threadIdx.x], r);
+      merge_ml(ml.x, ml.y, o.x, o.y);
+    }
+    const int row = q0 + threadIdx.x;
+    if (row < Lq) lse2[(size_t)h * Lq + row] = ml.x + log2f(ml.y);
+  }
+  cluster.sync();  // no CTA leaves while CTA 0 may still read its shared memory
 }
 
 template <typename T, int D>
@@ -137,11 +170,16 @@ __global__ void __launch_bounds__(kThreads)
   float* Ks = sm;
   float* Qs = sm + D * kPad;
   float* sl = sm + 2 * D * kPad;  // [64] row normalisers of the query tile
-  const int h = blockIdx.y, k0 = blockIdx.x * kT;
+  __shared__ float s_col[kT];     // this CTA's column sums of the key tile
+  cg::cluster_group cluster = cg::this_cluster();
+  const int nr = (int)cluster.num_blocks(), rank = (int)cluster.block_rank();
+  const int h = blockIdx.y, k0 = (blockIdx.x / nr) * kT;
   const int ty = threadIdx.x / 16, tx = threadIdx.x % 16;
+  const int nqt = (int)ceil_div(Lq, kT), per = (int)ceil_div(nqt, nr);
+  const int qt0 = rank * per, qt1 = min(nqt, qt0 + per);
   load_tile_t<T, D>(Ks, k + ((size_t)h * ldk + k0) * D, min(kT, Lk - k0));
   float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  for (int q0 = 0; q0 < Lq; q0 += kT) {
+  for (int q0 = qt0 * kT; q0 < qt1 * kT; q0 += kT) {
     __syncthreads();
     load_tile_t<T, D>(Qs, q + ((size_t)h * Lq + q0) * D, min(kT, Lq - q0));
     if (threadIdx.x < kT) {
@@ -167,9 +205,43 @@ __global__ void __launch_bounds__(kThreads)
     float t = 0.0f;
 #pragma unroll
     for (int y = 0; y < 16; ++y) t += red[y * kT + threadIdx.x];
+    s_col[threadIdx.x] = t;
+  }
+  cluster.sync();
+  // CTA 0 adds the cluster's query shares of each key, in rank order.
+  if (rank == 0 && threadIdx.x < kT) {
+    float t = s_col[threadIdx.x];
+    for (int r = 1; r < nr; ++r) t += *cluster.map_shared_rank(&s_col[threadIdx.x], r);
     const int key = k0 + threadIdx.x;
     if (key < Lk) imp[(size_t)h * Lk + key] = t / (float)Lq;
   }
+  cluster.sync();  // no CTA leaves while CTA 0 may still read its shared memory
+}
+
+// CTAs per cluster for `units` (tile, head) pairs each splittable into `tiles`
+// shares: enough to give about two CTAs per SM, at most 8 (the portable
+// cluster size) and at most one share per tile.
+int cluster_split(int64_t units, int tiles) {
+  const int64_t want = ceil_div(2 * (int64_t)sm_count(), units);
+  return (int)std::max<int64_t>(1, std::min<int64_t>({want, (int64_t)tiles, 8}));
+}
+
+template <typename K, typename... Args>
+cudaError_t launch_clustered(K kern, int nx, int H, int csize, size_t smem, cudaStream_t s,
+                             Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(nx * csize), (unsigned)H, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)csize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
 }
 
 template <typename T, int D>
@@ -178,14 +250,20 @@ cudaError_t run(const T* q, const T* k, int H, int Lq, int Lk, int ldk, float sc
   const float c2 = scale * kLog2e;
   const size_t smem1 = (size_t)2 * D * kPad * sizeof(float);
   const size_t smem2 = smem1 + kT * sizeof(float);
-  cudaFuncSetAttribute(imp_lse_simt<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)smem1);
-  cudaFuncSetAttribute(imp_col_simt<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       (int)smem2);
-  imp_lse_simt<T, D><<<dim3((unsigned)ceil_div(Lq, kT), H), kThreads, smem1, s>>>(q, k, Lq, Lk,
-                                                                                  ldk, c2, lse2);
-  imp_col_simt<T, D><<<dim3((unsigned)ceil_div(Lk, kT), H), kThreads, smem2, s>>>(
-      q, k, lse2, Lq, Lk, ldk, c2, imp);
+  cudaError_t e = cudaFuncSetAttribute(imp_lse_simt<T, D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(imp_col_simt<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem2);
+  if (e != cudaSuccess) return e;
+  const int nqt = (int)ceil_div(Lq, kT), nkt = (int)ceil_div(Lk, kT);
+  const int c1 = cluster_split((int64_t)nqt * H, nkt);
+  const int cc2 = cluster_split((int64_t)nkt * H, nqt);
+  e = launch_clustered(imp_lse_simt<T, D>, nqt, H, c1, smem1, s, q, k, Lq, Lk, ldk, c2, lse2);
+  if (e != cudaSuccess) return e;
+  e = launch_clustered(imp_col_simt<T, D>, nkt, H, cc2, smem2, s, q, k, (const float*)lse2, Lq,
+                       Lk, ldk, c2, imp);
+  if (e != cudaSuccess) return e;
   add_launches(2);
   return cudaGetLastError();
 }
