@@ -200,6 +200,26 @@ def test_score_topb_ties_and_signed_zero():
         np.testing.assert_array_equal(sc.view(np.uint32), sc_ref.view(np.uint32))
 
 
+@pytest.mark.parametrize("Lk", [65536, 131072, 196608])
+def test_score_topb_long_heads_mass_ties(Lk):
+    """Long heads (one 16-CTA cluster per head, the keys written over the
+    pooling tile) where most scores are equal: far more keys than the
+    candidate buffer holds share the threshold's top 16 bits, so the last two
+    radix passes scan the whole slice; the threshold falls inside the tie."""
+    H, B = 3, Lk // 4
+    rng = np.random.default_rng(Lk)
+    imp = np.full((H, Lk), 1.0 / Lk, np.float32)
+    red = np.full((H, Lk), 1.0 / Lk, np.float32)
+    imp[0, rng.choice(Lk, Lk // 16, replace=False)] = 2.0 / Lk  # pooled: ~40% above the tie
+    red[1, rng.choice(Lk, Lk // 2, replace=False)] = 0.5 / Lk   # half above, half tied
+    # head 2: every score ties; the B lowest indices are kept
+    sc_ref, idx_ref = O.score_topb(imp, red, 0.5, 7, B)
+    sc, idx = score_topb_gpu(imp, red, 7, 0.5, B)
+    np.testing.assert_array_equal(sc.view(np.uint32), sc_ref.view(np.uint32))
+    np.testing.assert_array_equal(idx, idx_ref)
+    np.testing.assert_array_equal(idx[2], np.arange(B, dtype=np.int32))
+
+
 @pytest.mark.parametrize("Lk,B", [(131072, 32768), (65536, 16384), (32760, 16380)])
 def test_score_topb_full_size_exact(Lk, B):
     """Full per-layer sizes (40 heads), including the case whose keys do not
